@@ -1,0 +1,183 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 linear layer.
+ *
+ * The layer (SVDQuant review, §4.2, low-rank decomposition equation):
+ *
+ *     Y = Q(X_hat) Q(R)  +  (X_hat L1) L2  +  bias,     X_hat = X diag(s)^-1
+ *
+ * with the low-rank branch fused into the 4-bit branch as in §4.3 (Nunchaku):
+ * the down-projection X_hat L1 is computed inside the activation-quantization
+ * kernel and the up-projection (X_hat L1) L2 inside the 4-bit GEMM.
+ * The offline decomposition (smoothing factors s, L1, L2, residual R) is
+ * computed by the caller and passed in as data ("From SmoothQuant to
+ * SVDQuant", section quantization scheme: weight-side quantities are static).
+ *
+ * Number formats (NVFP4, "From SmoothQuant to SVDQuant", section Personal view:
+ * groups of 16 with a two-level scale; SVDQuant review §3: q_max = 6):
+ *   - 4-bit codes are FP4 E2M1, two per byte along K, element 2j in the low
+ *     nibble of byte j.  An M x K operand is stored as M rows of K/2 bytes.
+ *   - one UE4M3 (unsigned E4M3) scale per 16 consecutive values along K,
+ *     stored in the "MMA scale order" below; one float32 global scale per
+ *     tensor, gs = amax / 2688 (1 when amax = 0).
+ *   - per group: sb = UE4M3_rne_sat(amax_group * f32(1 / f32(6 gs))),
+ *     d = f32(dec(sb) * gs), code = E2M1_rne_sat(x * f32(1/d)), all codes 0
+ *     when sb = 0.  Every step is one correctly rounded float32 operation.
+ *   - 16-bit tensors (X, L1f, L2, LAs, L2p, bias, bf16 Y) are bfloat16,
+ *     passed as uint16_t bit patterns.
+ *
+ * MMA scale order (the byte order the block-scaled tcgen05 MMA consumes):
+ * for an operand with `rows` rows and KS = K/16 scales per row, the buffer
+ * has svdq_sf_bytes(rows, K) = ceil(rows/128)*128*KS bytes; scale (r, kk)
+ * is at byte  ((r/128)*(KS/4) + kk/4)*512 + (r%32)*16 + ((r/32)%4)*4 + kk%4.
+ * Bytes of padding rows (rows..ceil(rows/128)*128-1) are written as 0 by
+ * the kernels that produce the buffer.
+ *
+ * Conventions for every call:
+ *   - Pointers are device pointers unless stated; the caller owns and
+ *     allocates every buffer; the library allocates no device memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Argument errors are returned before any launch;
+ *     a launch failure returns SVDQ_ERR_CUDA.  Kernel-side faults that do not
+ *     stop the kernel (a bounded wait that ran out) are reported by
+ *     svdq_get_device_error().
+ *   - Pointers must be 16-byte aligned.  Shapes: K % 64 == 0, N % 16 == 0,
+ *     r % 16 == 0 with 0 <= r <= 128, 1 <= M, K, N < 2^31.  Any M.
+ *   - One device per call: the current device of the calling thread.
+ *     Requires compute capability 10.0 (B200, sm_100a).
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SVDQ_API __attribute__((visibility("default")))
+#else
+#define SVDQ_API
+#endif
+
+typedef struct CUstream_st* svdq_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+    SVDQ_OK = 0,
+    SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad flag          */
+    SVDQ_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 64, N % 16, r % 16, r > 128, size overflow */
+    SVDQ_ERR_MISALIGNED = 3,         /* a pointer not 16-byte aligned                  */
+    SVDQ_ERR_CUDA = 4,               /* a CUDA runtime/driver call or launch failed    */
+    SVDQ_ERR_TIMEOUT = 5,            /* a kernel's bounded wait ran out (device error) */
+    SVDQ_ERR_DEVICE = 6              /* current device is not compute capability 10.x  */
+} svdq_status;
+
+/* Human-readable name of a status code (static string). */
+SVDQ_API const char* svdq_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+SVDQ_API int svdq_version(void);
+
+/* Bytes of a scale-factor buffer for a rows x K operand in MMA scale order
+ * (0 if rows < 0 or K % 64 != 0). */
+SVDQ_API size_t svdq_sf_bytes(int64_t rows, int64_t K);
+
+/*
+ * svdq_pack_weight -- static NVFP4 quantization of the residual weight
+ * (SVDQuant review, §4.2: only the residual R is quantized to 4 bits;
+ * "From SmoothQuant to SVDQuant", quantization scheme item 1: done offline).
+ *
+ *   R    [in]  float32, K x N row-major (N contiguous), finite values.
+ *   L2b  [in]  bf16, r x N row-major: the up-projection factor L2 (may be
+ *              NULL when r == 0).
+ *   Wq   [out] uint8, N x K/2: E2M1 codes of R^T (row n holds column n of R).
+ *   SFw  [out] uint8, svdq_sf_bytes(N, K): UE4M3 scales in MMA scale order.
+ *   gs_w [out] float32 (one device float): the weight global scale,
+ *              amax(|R|) / 2688; also used as the amax accumulator while the
+ *              call runs, so it must not alias anything else.
+ *   L2p  [out] bf16, N x 2r row-major: row n = [L2b[:, n] , L2b[:, n]], the
+ *              up-projection laid out K-major for the GEMM, doubled so that
+ *              the high and low halves of LAs (see svdq_quantize_act) meet
+ *              the same factor (NULL when r == 0).
+ * Four launches (zero, amax, scale, encode).  The caller reads gs_w back to
+ * form lr_scale for svdq_quantize_act.
+ */
+SVDQ_API svdq_status svdq_pack_weight(const float* R, const uint16_t* L2b, int64_t K, int64_t N, int r,
+                             uint8_t* Wq, uint8_t* SFw, float* gs_w, uint16_t* L2p,
+                             svdq_stream_t stream);
+
+/*
+ * svdq_quantize_act -- activation kernel with the fused down-projection
+ * (SVDQuant review, §4.3: the down-projection is merged into the
+ * quantization kernel so the activations are read once).
+ *
+ *   X        [in]  bf16, M x K row-major (read from HBM exactly once).
+ *   inv_s    [in]  float32, K: reciprocal smoothing factors 1/s_j;
+ *                  X_hat = f32(X * inv_s) (the smoothing divide).
+ *   gs_x     [in]  host float: static activation global scale (calibration).
+ *   L1fT     [in]  bf16, r x K row-major (K contiguous): (diag(s)^-1 L1)^T,
+ *                  the down factor with the smoothing folded in, so that
+ *                  X_hat L1 = X L1f.  May be NULL when r == 0.
+ *   lr_scale [in]  host float: f32(1 / (gs_x * gs_w)); the low-rank output
+ *                  is pre-scaled by it so the GEMM can add both branches in
+ *                  one accumulator and scale once by gs_x * gs_w.
+ *   Xq       [out] uint8, M x K/2: E2M1 codes of X_hat.
+ *   SFx      [out] uint8, svdq_sf_bytes(M, K): UE4M3 scales, MMA scale order.
+ *   LAs      [out] bf16, M x 2r: row m = [hi(v) | lo(v)] with
+ *                  v = f32(lr_scale * (X L1f)[m, :]) (fp32 accumulation),
+ *                  hi = bf16_rne(v), lo = bf16_rne(v - hi).  NULL when r == 0.
+ */
+SVDQ_API svdq_status svdq_quantize_act(const uint16_t* X, int64_t M, int64_t K, const float* inv_s,
+                              float gs_x, const uint16_t* L1fT, int r, float lr_scale,
+                              uint8_t* Xq, uint8_t* SFx, uint16_t* LAs, svdq_stream_t stream);
+
+/*
+ * svdq_linear -- block-scaled NVFP4 GEMM on the tcgen05 tensor cores with the
+ * up-projection fused into the same TMEM accumulator (SVDQuant review, §4.3:
+ * the up-projection is merged into the 4-bit GEMM kernel):
+ *
+ *   acc  = sum_k dec(Xq) dec(SFx) dec(Wq) dec(SFw)  +  LAs . L2p^T
+ *   Y    = f32(gs_x * gs_w) * acc + bias             (rounded once to bf16, or fp32)
+ *
+ *   Xq, SFx     [in] from svdq_quantize_act;  Wq, SFw, L2p [in] from svdq_pack_weight.
+ *   gs_x, gs_w  [in] host floats.
+ *   LAs, L2p    [in] may be NULL when r == 0 (plain NVFP4 GEMM).
+ *   bias        [in] bf16, N, or NULL.
+ *   Y           [out] M x N row-major: bf16 when y_fp32 == 0, float32 when 1.
+ * Persistent, warp-specialised kernel: one CTA per SM, 128 x 256 output tiles.
+ */
+SVDQ_API svdq_status svdq_linear(const uint8_t* Xq, const uint8_t* SFx, float gs_x,
+                        const uint8_t* Wq, const uint8_t* SFw, float gs_w,
+                        const uint16_t* LAs, const uint16_t* L2p, int r,
+                        const uint16_t* bias, void* Y, int y_fp32,
+                        int64_t M, int64_t N, int64_t K, svdq_stream_t stream);
+
+/*
+ * svdq_get_device_error -- synchronises `stream`, then reads and clears the
+ * library's device error word on the current device.  Returns SVDQ_OK, or
+ * SVDQ_ERR_TIMEOUT when a kernel's bounded wait on a barrier ran out (the
+ * kernel then stopped early; its outputs are undefined), or SVDQ_ERR_CUDA.
+ * If `site` is not NULL it receives an identifier of the wait that ran out.
+ */
+SVDQ_API svdq_status svdq_get_device_error(svdq_stream_t stream, int* site);
+
+/*
+ * svdq_linear_debug -- svdq_linear with test hooks, for the fault-path tests.
+ *   debug_flags bit 0: the load warp issues no loads, so the MMA warp's first
+ *                      wait can never complete and must run out.
+ *   timeout_ns: bound of every barrier wait (0 = the default of 2 s).
+ * Otherwise identical to svdq_linear.
+ */
+SVDQ_API svdq_status svdq_linear_debug(const uint8_t* Xq, const uint8_t* SFx, float gs_x,
+                              const uint8_t* Wq, const uint8_t* SFw, float gs_w,
+                              const uint16_t* LAs, const uint16_t* L2p, int r,
+                              const uint16_t* bias, void* Y, int y_fp32,
+                              int64_t M, int64_t N, int64_t K,
+                              int debug_flags, uint64_t timeout_ns, svdq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

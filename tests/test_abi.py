@@ -1,0 +1,78 @@
+"""The C ABI library loads, exports every declared symbol and validates arguments (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w4a4_rank_absorbed_b200 import build, svdq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return svdq.load_library()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    return sorted(set(re.findall(r"SVDQ_API\s+[\w\s\*]+?\b(svdq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert _declared() == sorted(svdq.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_sizes(lib):
+    assert svdq.status_string(0) == "SVDQ_OK"
+    assert svdq.status_string(5) == "SVDQ_ERR_TIMEOUT"
+    assert svdq.svdq_version() >= 100
+    assert svdq.svdq_sf_bytes(256, 512) == 256 * 32
+    assert svdq.svdq_sf_bytes(200, 512) == 256 * 32
+    assert svdq.svdq_sf_bytes(1, 64) == 128 * 4
+    assert svdq.svdq_sf_bytes(10, 100) == 0
+
+
+def _linear(lib, **kw):
+    a = dict(Xq=16, SFx=16, gs_x=1.0, Wq=16, SFw=16, gs_w=1.0, LAs=16, L2p=16, r=32, bias=None, Y=16,
+             y_fp32=0, M=128, N=256, K=256, stream=None)
+    a.update(kw)
+    return lib.svdq_linear(a["Xq"], a["SFx"], a["gs_x"], a["Wq"], a["SFw"], a["gs_w"], a["LAs"], a["L2p"],
+                           a["r"], a["bias"], a["Y"], a["y_fp32"], a["M"], a["N"], a["K"], a["stream"])
+
+
+def test_argument_errors_before_any_launch(lib):
+    assert _linear(lib, K=96) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert _linear(lib, N=24) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert _linear(lib, r=8) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert _linear(lib, r=144) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert _linear(lib, M=0) == svdq.SVDQ_ERR_INVALID_ARG
+    assert _linear(lib, M=1 << 31) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert _linear(lib, Xq=None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert _linear(lib, LAs=None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert _linear(lib, LAs=None, L2p=None, r=0) != svdq.SVDQ_ERR_INVALID_ARG
+    assert _linear(lib, y_fp32=2) == svdq.SVDQ_ERR_INVALID_ARG
+    assert _linear(lib, Y=24) == svdq.SVDQ_ERR_MISALIGNED
+    assert _linear(lib, bias=8) == svdq.SVDQ_ERR_MISALIGNED
+    assert lib.svdq_quantize_act(16, 64, 100, 16, 1.0, 16, 32, 1.0, 16, 16, 16, None) == \
+        svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert lib.svdq_quantize_act(16, 64, 128, 16, 1.0, None, 32, 1.0, 16, 16, 16, None) == \
+        svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_pack_weight(16, 16, 128, 40, 32, 16, 16, 16, 16, None) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert lib.svdq_pack_weight(4, 16, 128, 32, 32, 16, 16, 16, 16, None) == svdq.SVDQ_ERR_MISALIGNED
+    assert lib.svdq_linear_debug(16, 16, 1.0, 16, 16, 1.0, 16, 16, 32, None, 16, 0, 128, 256, 256, 4, 0, None) == \
+        svdq.SVDQ_ERR_INVALID_ARG
+
+
+def test_valid_arguments_without_a_gpu_report_a_device_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _linear(lib) in (svdq.SVDQ_ERR_CUDA, svdq.SVDQ_ERR_DEVICE)

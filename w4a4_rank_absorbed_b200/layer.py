@@ -1,0 +1,91 @@
+"""SVDQLinear: a packed SVDQuant W4A4 linear layer on one B200.
+
+Holds the packed residual weight and the low-rank factors in device memory
+and runs the forward pass as two launches of the CUDA library
+(SVDQuant review §4.3: down-projection fused into the quantization kernel,
+up-projection fused into the 4-bit GEMM):
+
+    svdq_quantize_act   X (bf16)  ->  Xq, SFx, LAs
+    svdq_linear         Xq, SFx, Wq, SFw, LAs, L2p, bias  ->  Y
+
+torch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import svdq as _C
+from .calib import LayerData
+
+
+def _f32(x) -> float:
+    return float(np.float32(x))
+
+
+class SVDQLinear:
+    def __init__(self, data: LayerData, device: Optional[torch.device] = None, stream=None):
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        self.K, self.N, self.r = data.K, data.N, data.r
+        self.gs_x = _f32(data.gs_x)
+        K, N, r = self.K, self.N, self.r
+        with torch.cuda.device(dev):
+            R = data.R.to(dev, torch.float32).contiguous()
+            L2b = data.L2b.to(dev).contiguous() if r else None
+            self.Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+            self.SFw = torch.empty(_C.svdq_sf_bytes(N, K), dtype=torch.uint8, device=dev)
+            self.gs_w_dev = torch.empty(1, dtype=torch.float32, device=dev)
+            self.L2p = torch.empty((N, 2 * r), dtype=torch.bfloat16, device=dev) if r else None
+            _C.svdq_pack_weight(R, L2b, K, N, r, self.Wq, self.SFw, self.gs_w_dev, self.L2p, stream)
+            self.gs_w = _f32(self.gs_w_dev.item())     # synchronises the stream
+            del R, L2b
+            self.inv_s = data.inv_s.to(dev, torch.float32).contiguous()
+            self.L1fT = data.L1fT.to(dev).contiguous() if r else None
+            self.bias = data.bias.to(dev).contiguous() if data.bias is not None else None
+        self.lr_scale = _f32(1.0 / (np.float64(self.gs_x) * np.float64(self.gs_w)))
+        self._act: Dict[int, tuple] = {}
+
+    def act_buffers(self, M: int):
+        """Device buffers of the quantized activations for M rows (allocated once per M)."""
+        if M not in self._act:
+            K, r, dev = self.K, self.r, self.device
+            self._act[M] = (torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                            torch.empty(_C.svdq_sf_bytes(M, K), dtype=torch.uint8, device=dev),
+                            torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev) if r else None)
+        return self._act[M]
+
+    def quantize(self, X: torch.Tensor, stream=None):
+        M = X.shape[0]
+        Xq, SFx, LAs = self.act_buffers(M)
+        _C.svdq_quantize_act(X, M, self.K, self.inv_s, self.gs_x, self.L1fT, self.r, self.lr_scale,
+                             Xq, SFx, LAs, stream)
+        return Xq, SFx, LAs
+
+    def gemm(self, Xq, SFx, LAs, Y: torch.Tensor, stream=None):
+        M = Xq.shape[0]
+        _C.svdq_linear(Xq, SFx, self.gs_x, self.Wq, self.SFw, self.gs_w, LAs, self.L2p, self.r, self.bias,
+                       Y, 1 if Y.dtype == torch.float32 else 0, M, self.N, self.K, stream)
+        return Y
+
+    def forward(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, y_fp32: bool = False,
+                stream=None) -> torch.Tensor:
+        """Y = layer(X); X bf16 [M, K] on the device; returns bf16 (or fp32) [M, N]."""
+        if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != self.K:
+            raise ValueError("X must be bf16 [M, K]")
+        M = X.shape[0]
+        if out is None:
+            out = torch.empty((M, self.N), dtype=torch.float32 if y_fp32 else torch.bfloat16, device=self.device)
+        Xq, SFx, LAs = self.quantize(X, stream)
+        return self.gemm(Xq, SFx, LAs, out, stream)
+
+    __call__ = forward
+
+    def forward_host(self, X_host: torch.Tensor, Y_host: torch.Tensor, X_dev: torch.Tensor,
+                     Y_dev: torch.Tensor) -> None:
+        """End-to-end call with host buffers: H2D of X, the two kernels, D2H of Y (asynchronous)."""
+        X_dev.copy_(X_host, non_blocking=True)
+        self.forward(X_dev, out=Y_dev)
+        Y_host.copy_(Y_dev, non_blocking=True)

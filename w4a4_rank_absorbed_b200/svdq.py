@@ -1,0 +1,160 @@
+"""Python binding of the C ABI in include/svdq.h (argument marshalling only).
+
+Each function has the name of the C entry point it calls and forwards torch
+CUDA tensors as raw device pointers; every step of the layer runs in the
+CUDA library ``libsvdq.so`` built in-tree by ``w4a4_rank_absorbed_b200.build``.
+There is no fallback: if the library is missing or the device is not an
+sm_100 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libsvdq.so")
+
+SVDQ_OK = 0
+SVDQ_ERR_INVALID_ARG = 1
+SVDQ_ERR_UNSUPPORTED_SHAPE = 2
+SVDQ_ERR_MISALIGNED = 3
+SVDQ_ERR_CUDA = 4
+SVDQ_ERR_TIMEOUT = 5
+SVDQ_ERR_DEVICE = 6
+
+EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_weight", "svdq_quantize_act",
+            "svdq_linear", "svdq_get_device_error", "svdq_linear_debug")
+
+
+class SVDQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_F = ctypes.c_float
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libsvdq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"CUDA library not built: {path} (run python -m w4a4_rank_absorbed_b200.build)")
+    lib = ctypes.CDLL(path)
+    lib.svdq_status_string.restype = ctypes.c_char_p
+    lib.svdq_status_string.argtypes = [_I]
+    lib.svdq_version.restype = _I
+    lib.svdq_version.argtypes = []
+    lib.svdq_sf_bytes.restype = ctypes.c_size_t
+    lib.svdq_sf_bytes.argtypes = [_I64, _I64]
+    lib.svdq_pack_weight.restype = _I
+    lib.svdq_pack_weight.argtypes = [_P, _P, _I64, _I64, _I, _P, _P, _P, _P, _P]
+    lib.svdq_quantize_act.restype = _I
+    lib.svdq_quantize_act.argtypes = [_P, _I64, _I64, _P, _F, _P, _I, _F, _P, _P, _P, _P]
+    lib.svdq_linear.restype = _I
+    lib.svdq_linear.argtypes = [_P, _P, _F, _P, _P, _F, _P, _P, _I, _P, _P, _I, _I64, _I64, _I64, _P]
+    lib.svdq_linear_debug.restype = _I
+    lib.svdq_linear_debug.argtypes = [_P, _P, _F, _P, _P, _F, _P, _P, _I, _P, _P, _I, _I64, _I64, _I64, _I,
+                                      ctypes.c_uint64, _P]
+    lib.svdq_get_device_error.restype = _I
+    lib.svdq_get_device_error.argtypes = [_P, ctypes.POINTER(_I)]
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().svdq_status_string(int(status)).decode()
+    except ImportError:
+        return f"status {status}"
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name: str = "") -> Optional[int]:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, where: str):
+    if status != SVDQ_OK:
+        raise SVDQError(status, where)
+
+
+def svdq_sf_bytes(rows: int, K: int) -> int:
+    return int(load_library().svdq_sf_bytes(rows, K))
+
+
+def svdq_version() -> int:
+    return int(load_library().svdq_version())
+
+
+def svdq_pack_weight(R, L2b, K, N, r, Wq, SFw, gs_w, L2p, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_pack_weight(_ptr(R, torch.float32, "R"), _ptr(L2b, torch.bfloat16, "L2b"), K, N, r,
+                              _ptr(Wq, torch.uint8, "Wq"), _ptr(SFw, torch.uint8, "SFw"),
+                              _ptr(gs_w, torch.float32, "gs_w"), _ptr(L2p, torch.bfloat16, "L2p"), _stream(stream))
+    _check(st, "svdq_pack_weight")
+
+
+def svdq_quantize_act(X, M, K, inv_s, gs_x, L1fT, r, lr_scale, Xq, SFx, LAs, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_quantize_act(_ptr(X, torch.bfloat16, "X"), M, K, _ptr(inv_s, torch.float32, "inv_s"),
+                               float(gs_x), _ptr(L1fT, torch.bfloat16, "L1fT"), r, float(lr_scale),
+                               _ptr(Xq, torch.uint8, "Xq"), _ptr(SFx, torch.uint8, "SFx"),
+                               _ptr(LAs, torch.bfloat16, "LAs"), _stream(stream))
+    _check(st, "svdq_quantize_act")
+
+
+def svdq_linear(Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p, r, bias, Y, y_fp32, M, N, K, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_linear(_ptr(Xq, torch.uint8, "Xq"), _ptr(SFx, torch.uint8, "SFx"), float(gs_x),
+                         _ptr(Wq, torch.uint8, "Wq"), _ptr(SFw, torch.uint8, "SFw"), float(gs_w),
+                         _ptr(LAs, torch.bfloat16, "LAs"), _ptr(L2p, torch.bfloat16, "L2p"), r,
+                         _ptr(bias, torch.bfloat16, "bias"), _ptr(Y, (torch.bfloat16, torch.float32), "Y"),
+                         int(y_fp32), M, N, K, _stream(stream))
+    _check(st, "svdq_linear")
+
+
+def svdq_linear_debug(Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p, r, bias, Y, y_fp32, M, N, K, debug_flags,
+                      timeout_ns, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_linear_debug(_ptr(Xq, torch.uint8, "Xq"), _ptr(SFx, torch.uint8, "SFx"), float(gs_x),
+                               _ptr(Wq, torch.uint8, "Wq"), _ptr(SFw, torch.uint8, "SFw"), float(gs_w),
+                               _ptr(LAs, torch.bfloat16, "LAs"), _ptr(L2p, torch.bfloat16, "L2p"), r,
+                               _ptr(bias, torch.bfloat16, "bias"), _ptr(Y, (torch.bfloat16, torch.float32), "Y"),
+                               int(y_fp32), M, N, K, int(debug_flags), int(timeout_ns), _stream(stream))
+    _check(st, "svdq_linear_debug")
+
+
+def svdq_get_device_error(stream=None):
+    """Returns (status, site); clears the device error word."""
+    lib = load_library()
+    site = _I(0)
+    st = lib.svdq_get_device_error(_stream(stream), ctypes.byref(site))
+    return int(st), int(site.value)
