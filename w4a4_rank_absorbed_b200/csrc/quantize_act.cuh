@@ -9,32 +9,44 @@
 // diag(s)^-1 L1, so X L1f = X_hat L1) on the tensor cores (bf16 in, fp32
 // accumulate), pre-scaled by lr_scale and split into bf16 hi/lo halves.
 //
-// CTA = 32 rows x all of K; 8 consumer warps + 1 TMA producer warp.
-// Stage = one 64-column chunk: X box 32 x 64 bf16 (4 KB) and L1f^T box
-// r x 64 bf16, both 128-byte swizzled.  Consumer thread t handles row t/8,
-// columns 8(t%8)..+7 of the chunk (half a group; the pair of threads of a
-// group combine their maxima with one shuffle).  Warp w owns the (16-row,
-// 8-column) tiles p = w, w+8, ... of the 32 x r down-projection output and
-// keeps them in registers across the whole K loop (mma.sync m16n8k16).
+// CTA = 32 rows x all of K; 7 consumer warps + 1 TMA producer warp (8 warps: two per
+// SM sub-partition, so each thread may hold up to 255 registers).
+// The K axis is cut into 64-column chunks; chunk c goes through ring stage
+// c % S and is consumed by warp c % 7 alone, so seven chunks are processed
+// at once and up to S loads are in flight.  A stage holds the X box
+// (32 x 64 bf16, 128-byte swizzle), the L1f^T box (r x 64 bf16, same
+// swizzle) and the 64 smoothing factors of the chunk.  In a chunk, lane l
+// quantizes row l (four groups of 16) and the warp runs the whole 32 x r
+// down-projection for the chunk's 64 columns (mma.sync m16n8k16), keeping
+// a partial sum in registers.  After the last chunk the seven partial sums
+// are added in shared memory and written as LAs.
 #pragma once
 #include "common.cuh"
 
 namespace svdq {
 
 constexpr int QA_ROWS = 32;
-constexpr int QA_CHUNK = 64;          // bf16 columns per stage (128 bytes)
-constexpr int QA_CONSUMER_WARPS = 8;
+constexpr int QA_CHUNK = 64;          // bf16 columns per chunk (128 bytes)
+constexpr int QA_CONSUMER_WARPS = 7;
 constexpr int QA_THREADS = (QA_CONSUMER_WARPS + 1) * 32;
+constexpr int QA_RING_BYTES = 160 * 1024;
 
 template <int R>
 struct QaCfg {
-  static constexpr int kStages = R <= 32 ? 8 : (R <= 64 ? 6 : 4);
   static constexpr int kXBytes = QA_ROWS * 128;
   static constexpr int kLBytes = R * 128;
   static constexpr int kStageBytes = kXBytes + kLBytes;
-  static constexpr int kTiles = 2 * (R / 8);                        // (m16, n8) tiles of the 32 x R output
-  static constexpr int kTilesPerWarp = (kTiles + QA_CONSUMER_WARPS - 1) / QA_CONSUMER_WARPS;
-  static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8 + 16 + 1024;
+  static constexpr int kStagesFit = QA_RING_BYTES / kStageBytes;
+  static constexpr int kStages = kStagesFit < 16 ? kStagesFit : 16;
+  static constexpr int kNT = R / 8;                                  // n8 tiles of the r columns
+  static constexpr int kAcc = R > 0 ? 2 * kNT : 1;                  // (m16, n8) tiles per warp
+  static constexpr int kRedBytes = QA_CONSUMER_WARPS * QA_ROWS * R * 4;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static_assert(kRedBytes <= kRingBytes, "reduction buffer must fit in the ring");
+  static constexpr int kInvOff = kRingBytes;                        // S x 64 floats
+  static constexpr int kRcpOff = kInvOff + kStages * 256;           // 128-entry 1/d table
+  static constexpr int kBarOff = kRcpOff + 128 * 4;
+  static constexpr int kSmem = kBarOff + 2 * kStages * 8 + 16 + 1024;
 };
 
 SVDQ_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -53,22 +65,67 @@ SVDQ_DEV void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+SVDQ_DEV void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 // Byte offset of 16-byte chunk `c16` of row `row` in a 128-byte-swizzled tile.
 SVDQ_DEV uint32_t sw128(uint32_t row, uint32_t c16) { return row * 128u + ((c16 ^ (row & 7u)) << 4); }
 
+// One group of 16 values of X (two 16-byte smem chunks) times 16 smoothing factors:
+// returns the UE4M3 scale and the two 32-bit code words.
+SVDQ_DEV uint32_t quant_group(const uint4& r0, const uint4& r1, const float4* inv, float c_x,
+                              const float* rcp_table, uint32_t& w0, uint32_t& w1) {
+  const float4 s0 = inv[0], s1 = inv[1], s2 = inv[2], s3 = inv[3];
+  float xh[16];
+  xh[0] = __fmul_rn(bf16_lo(r0.x), s0.x);
+  xh[1] = __fmul_rn(bf16_hi(r0.x), s0.y);
+  xh[2] = __fmul_rn(bf16_lo(r0.y), s0.z);
+  xh[3] = __fmul_rn(bf16_hi(r0.y), s0.w);
+  xh[4] = __fmul_rn(bf16_lo(r0.z), s1.x);
+  xh[5] = __fmul_rn(bf16_hi(r0.z), s1.y);
+  xh[6] = __fmul_rn(bf16_lo(r0.w), s1.z);
+  xh[7] = __fmul_rn(bf16_hi(r0.w), s1.w);
+  xh[8] = __fmul_rn(bf16_lo(r1.x), s2.x);
+  xh[9] = __fmul_rn(bf16_hi(r1.x), s2.y);
+  xh[10] = __fmul_rn(bf16_lo(r1.y), s2.z);
+  xh[11] = __fmul_rn(bf16_hi(r1.y), s2.w);
+  xh[12] = __fmul_rn(bf16_lo(r1.z), s3.x);
+  xh[13] = __fmul_rn(bf16_hi(r1.z), s3.y);
+  xh[14] = __fmul_rn(bf16_lo(r1.w), s3.z);
+  xh[15] = __fmul_rn(bf16_hi(r1.w), s3.w);
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(xh[i]));
+  const uint32_t sb = cvt_ue4m3(__fmul_rn(a, c_x));
+  const float rinv = rcp_table[sb];           // f32(1 / f32(dec(sb) * gs)); entry 0 is 0
+  float q0[8], q1[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    q0[i] = __fmul_rn(xh[i], rinv);
+    q1[i] = __fmul_rn(xh[8 + i], rinv);
+  }
+  // rinv = 0 for an all-zero scale: every product is +-0; the codes are forced to 0.
+  w0 = sb ? cvt_e2m1x8(q0) : 0u;
+  w1 = sb ? cvt_e2m1x8(q1) : 0u;
+  return sb;
+}
+
 template <int R>
-__global__ void __launch_bounds__(QA_THREADS) k_quantize_act(
+__global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
     const __grid_constant__ CUtensorMap tm_x,   // bf16 {K, M}, box {64, 32}, 128B swizzle
     const __grid_constant__ CUtensorMap tm_l1,  // bf16 {K, R}, box {64, R}, 128B swizzle
     const float* __restrict__ inv_s, float gs_x, float lr_scale, int M, int K, int Mpad,
     uint8_t* __restrict__ Xq, uint8_t* __restrict__ SFx, uint16_t* __restrict__ LAs, uint64_t timeout_ns) {
   using Cfg = QaCfg<R>;
+  constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kStages * Cfg::kStageBytes);
-  uint64_t* empty = full + Cfg::kStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + Cfg::kStages);
+  float* s_inv = reinterpret_cast<float*>(smem + Cfg::kInvOff);
+  float* s_rcp = reinterpret_cast<float*>(smem + Cfg::kRcpOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* empty = full + S;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -76,12 +133,17 @@ __global__ void __launch_bounds__(QA_THREADS) k_quantize_act(
   const int nchunks = K / QA_CHUNK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < Cfg::kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], QA_CONSUMER_WARPS);
+      mbar_init(&empty[s], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  // 1/d for every possible block scale: d = f32(dec(sb) * gs_x), same operations as the per-group path.
+  if (threadIdx.x < 128) {
+    const uint32_t sb = threadIdx.x;
+    s_rcp[sb] = sb == 0 ? 0.0f : __frcp_rn(__fmul_rn(dec_ue4m3(sb), gs_x));
   }
   __syncthreads();
 
@@ -90,126 +152,131 @@ __global__ void __launch_bounds__(QA_THREADS) k_quantize_act(
     if (lane == 0) {
       tma_prefetch_desc(&tm_x);
       if (R > 0) tma_prefetch_desc(&tm_l1);
-      int stage = 0;
-      uint32_t phase = 0;
       for (int c = 0; c < nchunks; ++c) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, timeout_ns, abort_flag, 0x201)) break;
-        uint8_t* sx = smem + stage * Cfg::kStageBytes;
-        mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
-        tma_load_2d(sx, &tm_x, &full[stage], c * QA_CHUNK, m0);
-        if (R > 0) tma_load_2d(sx + Cfg::kXBytes, &tm_l1, &full[stage], c * QA_CHUNK, 0);
-        if (++stage == Cfg::kStages) { stage = 0; phase ^= 1u; }
+        const int s = c % S;
+        const uint32_t parity = (uint32_t)((c / S) & 1);
+        if (!mbar_wait(&empty[s], parity ^ 1u, timeout_ns, abort_flag, 0x201)) break;
+        uint8_t* st = smem + s * Cfg::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes + 256);
+        tma_load_2d(st, &tm_x, &full[s], c * QA_CHUNK, m0);
+        if (R > 0) tma_load_2d(st + Cfg::kXBytes, &tm_l1, &full[s], c * QA_CHUNK, 0);
+        bulk_load(s_inv + s * 64, inv_s + (int64_t)c * QA_CHUNK, 256, &full[s]);
       }
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers --
-  const int t = threadIdx.x;
-  const int row = t >> 3;            // 0..31
-  const int j = t & 7;               // 8-column slice of the 64-column chunk
-  const int m = m0 + row;
+  const int m = m0 + lane;                 // this lane's row for the quantizer
   const float c_x = __frcp_rn(__fmul_rn(6.0f, gs_x));
   const uint32_t KS4 = (uint32_t)(K >> 6);
-  const int64_t xq_row = (int64_t)m * (K >> 1);
 
-  float acc[Cfg::kTilesPerWarp > 0 ? Cfg::kTilesPerWarp : 1][4];
+  float acc[Cfg::kAcc][4];
 #pragma unroll
-  for (int i = 0; i < (Cfg::kTilesPerWarp > 0 ? Cfg::kTilesPerWarp : 1); ++i)
-    acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+  for (int i = 0; i < Cfg::kAcc; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
 
-  int stage = 0;
-  uint32_t phase = 0;
   bool ok = true;
-  for (int c = 0; c < nchunks; ++c) {
-    if (!mbar_wait(&full[stage], phase, timeout_ns, abort_flag, 0x202)) { ok = false; break; }
-    const uint8_t* sx = smem + stage * Cfg::kStageBytes;
-    const uint32_t sx_u32 = smem_u32(sx);
-
-    // ---- quantize 8 elements (half a group) -------------------------------
-    const int k0 = c * QA_CHUNK + 8 * j;
-    const uint4 raw = *reinterpret_cast<const uint4*>(sx + sw128(row, j));
-    const float4 s0 = __ldg(reinterpret_cast<const float4*>(inv_s + k0));
-    const float4 s1 = __ldg(reinterpret_cast<const float4*>(inv_s + k0 + 4));
-    float xh[8];
-    xh[0] = __fmul_rn(bf16_lo(raw.x), s0.x);
-    xh[1] = __fmul_rn(bf16_hi(raw.x), s0.y);
-    xh[2] = __fmul_rn(bf16_lo(raw.y), s0.z);
-    xh[3] = __fmul_rn(bf16_hi(raw.y), s0.w);
-    xh[4] = __fmul_rn(bf16_lo(raw.z), s1.x);
-    xh[5] = __fmul_rn(bf16_hi(raw.z), s1.y);
-    xh[6] = __fmul_rn(bf16_lo(raw.w), s1.z);
-    xh[7] = __fmul_rn(bf16_hi(raw.w), s1.w);
-    float a = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(xh[i]));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-    const uint32_t sb = cvt_ue4m3(__fmul_rn(a, c_x));
-    uint32_t code = 0u;
-    if (sb != 0u) {
-      const float rinv = __frcp_rn(__fmul_rn(dec_ue4m3(sb), gs_x));
-      float q[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(xh[i], rinv);
-      code = cvt_e2m1x8(q);
+  for (int c = warp; c < nchunks; c += QA_CONSUMER_WARPS) {
+    const int s = c % S;
+    if (!mbar_wait(&full[s], (uint32_t)((c / S) & 1), timeout_ns, abort_flag, 0x202)) {
+      ok = false;
+      break;
     }
-    if (m < M) *reinterpret_cast<uint32_t*>(Xq + xq_row + (k0 >> 1)) = code;
-    const uint32_t s2 = __shfl_down_sync(0xffffffffu, sb, 2);
-    const uint32_t s4 = __shfl_down_sync(0xffffffffu, sb, 4);
-    const uint32_t s6 = __shfl_down_sync(0xffffffffu, sb, 6);
-    if (j == 0 && m < Mpad)
-      *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)m, (uint32_t)c, KS4)) =
-          sb | (s2 << 8) | (s4 << 16) | (s6 << 24);
+    const uint8_t* st = smem + s * Cfg::kStageBytes;
+    const uint32_t st_u32 = smem_u32(st);
+    const float4* inv = reinterpret_cast<const float4*>(s_inv + s * 64);
 
-    // ---- down-projection on the tensor cores ------------------------------
+    // ---- quantize row `lane`: four groups of 16 ---------------------------
+    uint32_t w[8];
+    uint32_t sfword = 0u;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint4 r0 = *reinterpret_cast<const uint4*>(st + sw128(lane, 2 * g));
+      const uint4 r1 = *reinterpret_cast<const uint4*>(st + sw128(lane, 2 * g + 1));
+      const uint32_t sb = quant_group(r0, r1, inv + 4 * g, c_x, s_rcp, w[2 * g], w[2 * g + 1]);
+      sfword |= sb << (8 * g);
+    }
+    if (m < M) {
+      uint4* dst = reinterpret_cast<uint4*>(Xq + (int64_t)m * (K >> 1) + c * 32);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+    if (m < Mpad) *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)m, (uint32_t)c, KS4)) = sfword;
+
+    // ---- down-projection of the chunk on the tensor cores -----------------
     if constexpr (R > 0) {
-      const uint32_t sl_u32 = sx_u32 + Cfg::kXBytes;
+      const uint32_t sl_u32 = st_u32 + Cfg::kXBytes;
 #pragma unroll
-      for (int i = 0; i < Cfg::kTilesPerWarp; ++i) {
-        const int p = warp + QA_CONSUMER_WARPS * i;
-        if (p < Cfg::kTiles) {
-          const int mt = p / (R / 8);
-          const int nt = p % (R / 8);
+      for (int ks = 0; ks < 4; ++ks) {
+        uint32_t a[2][4];
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            uint32_t a0, a1, a2, a3, b0, b1;
-            const uint32_t arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            ldsm_x4(sx_u32 + sw128(arow, ks * 2 + (lane >> 4)), a0, a1, a2, a3);
+        for (int mt = 0; mt < 2; ++mt) {
+          const uint32_t arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          ldsm_x4(st_u32 + sw128(arow, ks * 2 + (lane >> 4)), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < Cfg::kNT; nt += 2) {
+          uint32_t b[4];
+          if (nt + 1 < Cfg::kNT) {
+            const uint32_t brow = (nt + (lane >> 4)) * 8 + (lane & 7);
+            ldsm_x4(sl_u32 + sw128(brow, ks * 2 + ((lane >> 3) & 1)), b[0], b[1], b[2], b[3]);
+          } else {
             const uint32_t brow = nt * 8 + (lane & 7);
-            ldsm_x2(sl_u32 + sw128(brow, ks * 2 + ((lane >> 3) & 1)), b0, b1);
-            mma_bf16_16816(acc[i], a0, a1, a2, a3, b0, b1);
+            ldsm_x2(sl_u32 + sw128(brow, ks * 2 + ((lane >> 3) & 1)), b[0], b[1]);
+            b[2] = b[3] = 0u;
+          }
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            mma_bf16_16816(acc[mt * Cfg::kNT + nt], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b[0], b[1]);
+            if (nt + 1 < Cfg::kNT)
+              mma_bf16_16816(acc[mt * Cfg::kNT + nt + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b[2], b[3]);
           }
         }
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
-    if (++stage == Cfg::kStages) { stage = 0; phase ^= 1u; }
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
 
-  // ---- LAs = [hi | lo] of lr_scale * (X L1f) -------------------------------
+  // ---- LAs = [hi | lo] of lr_scale * sum over warps of the partial X L1f ----
   if constexpr (R > 0) {
+    // Every chunk has been consumed, so no load is in flight into the ring: reuse it.
+    named_bar_sync(1, QA_CONSUMER_WARPS * 32);
+    float* red = reinterpret_cast<float*>(smem);            // [warp][row][R]
     if (ok) {
 #pragma unroll
-      for (int i = 0; i < Cfg::kTilesPerWarp; ++i) {
-        const int p = warp + QA_CONSUMER_WARPS * i;
-        if (p < Cfg::kTiles) {
-          const int mt = p / (R / 8);
-          const int nt = p % (R / 8);
-          const int col = nt * 8 + 2 * (lane & 3);
+      for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int mm = m0 + mt * 16 + (lane >> 2) + 8 * h;
-            if (mm < M) {
-              const float v0 = __fmul_rn(acc[i][2 * h], lr_scale);
-              const float v1 = __fmul_rn(acc[i][2 * h + 1], lr_scale);
-              const float h0 = __bfloat162float(__float2bfloat16_rn(v0));
-              const float h1 = __bfloat162float(__float2bfloat16_rn(v1));
-              uint16_t* dst = LAs + (int64_t)mm * (2 * R);
-              *reinterpret_cast<uint32_t*>(dst + col) = pack_bf16x2(h0, h1);
-              *reinterpret_cast<uint32_t*>(dst + R + col) = pack_bf16x2(v0 - h0, v1 - h1);
-            }
-          }
+        for (int nt = 0; nt < Cfg::kNT; ++nt) {
+          const int row = mt * 16 + (lane >> 2);
+          const int col = nt * 8 + 2 * (lane & 3);
+          float* p = red + ((warp * QA_ROWS + row) * R + col);
+          *reinterpret_cast<float2*>(p) = make_float2(acc[mt * Cfg::kNT + nt][0], acc[mt * Cfg::kNT + nt][1]);
+          *reinterpret_cast<float2*>(p + 8 * R) =
+              make_float2(acc[mt * Cfg::kNT + nt][2], acc[mt * Cfg::kNT + nt][3]);
+        }
+    }
+    named_bar_sync(1, QA_CONSUMER_WARPS * 32);
+    if (ok && !*abort_flag) {
+      for (int p = threadIdx.x; p < QA_ROWS * R / 2; p += QA_CONSUMER_WARPS * 32) {
+        const int row = p / (R / 2);
+        const int col = 2 * (p % (R / 2));
+        float v0 = 0.0f, v1 = 0.0f;
+#pragma unroll
+        for (int w2 = 0; w2 < QA_CONSUMER_WARPS; ++w2) {
+          const float2 t = *reinterpret_cast<const float2*>(red + ((w2 * QA_ROWS + row) * R + col));
+          v0 += t.x;
+          v1 += t.y;
+        }
+        const int mm = m0 + row;
+        if (mm < M) {
+          v0 = __fmul_rn(v0, lr_scale);
+          v1 = __fmul_rn(v1, lr_scale);
+          const float h0 = __bfloat162float(__float2bfloat16_rn(v0));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(v1));
+          uint16_t* dst = LAs + (int64_t)mm * (2 * R);
+          *reinterpret_cast<uint32_t*>(dst + col) = pack_bf16x2(h0, h1);
+          *reinterpret_cast<uint32_t*>(dst + R + col) = pack_bf16x2(v0 - h0, v1 - h1);
         }
       }
     }
