@@ -9,17 +9,17 @@
 // diag(s)^-1 L1, so X L1f = X_hat L1) on the tensor cores (bf16 in, fp32
 // accumulate), pre-scaled by lr_scale and split into bf16 hi/lo halves.
 //
-// CTA = 32 rows x all of K; 7 consumer warps + 1 TMA producer warp (8 warps: two per
-// SM sub-partition, so each thread may hold up to 255 registers).
+// CTA = 32 rows x all of K; 14 consumer warps in 7 pairs + 1 TMA producer warp.
 // The K axis is cut into 64-column chunks; chunk c goes through ring stage
-// c % S and is consumed by warp c % 7 alone, so seven chunks are processed
-// at once and up to S loads are in flight.  A stage holds the X box
-// (32 x 64 bf16, 128-byte swizzle), the L1f^T box (r x 64 bf16, same
-// swizzle) and the 64 smoothing factors of the chunk.  In a chunk, lane l
-// quantizes row l (four groups of 16) and the warp runs the whole 32 x r
-// down-projection for the chunk's 64 columns (mma.sync m16n8k16), keeping
-// a partial sum in registers.  After the last chunk the seven partial sums
-// are added in shared memory and written as LAs.
+// c % S and is consumed by warp pair c % 7, so seven chunks are processed at
+// once and up to S loads are in flight (S = 14, or 7 for r > 88; S is a multiple of 7).  A stage holds the X box (32 x 64
+// bf16, 128-byte swizzle) and the L1f^T box (r x 64 bf16, same swizzle); the
+// 64 smoothing factors of the chunk are read through the read-only cache.  Warp h of a pair owns rows 16h..16h+15
+// of the chunk: two lanes per row quantize two groups of 16 each, and the
+// warp runs the 16 x r down-projection of its rows for the chunk's 64 columns
+// (mma.sync m16n8k16), keeping a partial sum in registers.  After the last
+// chunk the seven partial sums of every row are added in shared memory and
+// written as LAs.
 #pragma once
 #include "common.cuh"
 
@@ -27,24 +27,26 @@ namespace svdq {
 
 constexpr int QA_ROWS = 32;
 constexpr int QA_CHUNK = 64;          // bf16 columns per chunk (128 bytes)
-constexpr int QA_CONSUMER_WARPS = 7;
+constexpr int QA_PAIRS = 7;
+constexpr int QA_CONSUMER_WARPS = 2 * QA_PAIRS;
 constexpr int QA_THREADS = (QA_CONSUMER_WARPS + 1) * 32;
-constexpr int QA_RING_BYTES = 160 * 1024;
+constexpr int QA_RING_BYTES = 200 * 1024;
 
 template <int R>
 struct QaCfg {
   static constexpr int kXBytes = QA_ROWS * 128;
   static constexpr int kLBytes = R * 128;
   static constexpr int kStageBytes = kXBytes + kLBytes;
-  static constexpr int kStagesFit = QA_RING_BYTES / kStageBytes;
-  static constexpr int kStages = kStagesFit < 16 ? kStagesFit : 16;
+  // The ring size is a multiple of the pair count, so a ring slot is always consumed by the
+  // same warp pair and its rounds are waited for in order (a parity wait cannot tell round r
+  // from round r - 2).
+  static constexpr int kStages = (2 * QA_PAIRS * kStageBytes <= QA_RING_BYTES) ? 2 * QA_PAIRS : QA_PAIRS;
   static constexpr int kNT = R / 8;                                  // n8 tiles of the r columns
-  static constexpr int kAcc = R > 0 ? 2 * kNT : 1;                  // (m16, n8) tiles per warp
-  static constexpr int kRedBytes = QA_CONSUMER_WARPS * QA_ROWS * R * 4;
+  static constexpr int kAcc = R > 0 ? kNT : 1;                      // (m16, n8) tiles per warp
+  static constexpr int kRedBytes = QA_PAIRS * QA_ROWS * R * 4;
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kRedBytes <= kRingBytes, "reduction buffer must fit in the ring");
-  static constexpr int kInvOff = kRingBytes;                        // S x 64 floats
-  static constexpr int kRcpOff = kInvOff + kStages * 256;           // 128-entry 1/d table
+  static constexpr int kRcpOff = kRingBytes;                        // 128-entry 1/d table
   static constexpr int kBarOff = kRcpOff + 128 * 4;
   static constexpr int kSmem = kBarOff + 2 * kStages * 8 + 16 + 1024;
 };
@@ -121,7 +123,6 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* s_inv = reinterpret_cast<float*>(smem + Cfg::kInvOff);
   float* s_rcp = reinterpret_cast<float*>(smem + Cfg::kRcpOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
   uint64_t* empty = full + S;
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 2);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -149,25 +150,34 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
 
   if (warp == QA_CONSUMER_WARPS) {
     // ---------------------------------------------------------- producer --
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_x);
-      if (R > 0) tma_prefetch_desc(&tm_l1);
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % S;
+    // Lane 2g + k serves ring slot g (chunks c with c % S == g) and stream k (0: X box,
+    // 1: L1f^T box).  A thread's TMA copies are serviced one after another, so each lane
+    // keeps at most one copy in flight.
+    const int g = lane >> 1, k = lane & 1;
+    if (g < S && (k == 0 || R > 0)) {
+      if (lane == 0) tma_prefetch_desc(&tm_x);
+      if (lane == 1) tma_prefetch_desc(&tm_l1);
+      for (int c = g; c < nchunks; c += S) {
         const uint32_t parity = (uint32_t)((c / S) & 1);
-        if (!mbar_wait(&empty[s], parity ^ 1u, timeout_ns, abort_flag, 0x201)) break;
-        uint8_t* st = smem + s * Cfg::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes + 256);
-        tma_load_2d(st, &tm_x, &full[s], c * QA_CHUNK, m0);
-        if (R > 0) tma_load_2d(st + Cfg::kXBytes, &tm_l1, &full[s], c * QA_CHUNK, 0);
-        bulk_load(s_inv + s * 64, inv_s + (int64_t)c * QA_CHUNK, 256, &full[s]);
+        if (!mbar_wait(&empty[g], parity ^ 1u, timeout_ns, abort_flag, 0x201)) break;
+        uint8_t* st = smem + g * Cfg::kStageBytes;
+        if (k == 0) {
+          mbar_arrive_expect_tx(&full[g], Cfg::kStageBytes);
+          tma_load_2d(st, &tm_x, &full[g], c * QA_CHUNK, m0);
+        } else {
+          tma_load_2d(st + Cfg::kXBytes, &tm_l1, &full[g], c * QA_CHUNK, 0);
+        }
       }
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers --
-  const int m = m0 + lane;                 // this lane's row for the quantizer
+  const int pairi = warp >> 1;             // warp pair: consumes chunks pairi, pairi + 7, ...
+  const int half = warp & 1;               // rows 16*half .. 16*half + 15 of the chunk
+  const int qrow = 16 * half + (lane >> 1);
+  const int qg = 2 * (lane & 1);           // first of the two groups this lane quantizes
+  const int m = m0 + qrow;
   const float c_x = __frcp_rn(__fmul_rn(6.0f, gs_x));
   const uint32_t KS4 = (uint32_t)(K >> 6);
 
@@ -176,61 +186,54 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   for (int i = 0; i < Cfg::kAcc; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
 
   bool ok = true;
-  for (int c = warp; c < nchunks; c += QA_CONSUMER_WARPS) {
+  for (int c = pairi; c < nchunks; c += QA_PAIRS) {
     const int s = c % S;
+    // smoothing factors of this lane's two groups (read-only path; issued before the wait)
+    float4 inv[8];
+    {
+      const float4* src = reinterpret_cast<const float4*>(inv_s + (int64_t)c * QA_CHUNK + 16 * qg);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) inv[i] = __ldg(src + i);
+    }
     if (!mbar_wait(&full[s], (uint32_t)((c / S) & 1), timeout_ns, abort_flag, 0x202)) {
       ok = false;
       break;
     }
     const uint8_t* st = smem + s * Cfg::kStageBytes;
     const uint32_t st_u32 = smem_u32(st);
-    const float4* inv = reinterpret_cast<const float4*>(s_inv + s * 64);
 
-    // ---- quantize row `lane`: four groups of 16 ---------------------------
-    uint32_t w[8];
-    uint32_t sfword = 0u;
+    // ---- quantize two groups of row qrow ------------------------------------
+    uint32_t w[4];
+    uint32_t sb2 = 0u;
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const uint4 r0 = *reinterpret_cast<const uint4*>(st + sw128(lane, 2 * g));
-      const uint4 r1 = *reinterpret_cast<const uint4*>(st + sw128(lane, 2 * g + 1));
+    for (int g = 0; g < 2; ++g) {
+      const int gg = qg + g;
+      const uint4 r0 = *reinterpret_cast<const uint4*>(st + sw128(qrow, 2 * gg));
+      const uint4 r1 = *reinterpret_cast<const uint4*>(st + sw128(qrow, 2 * gg + 1));
       const uint32_t sb = quant_group(r0, r1, inv + 4 * g, c_x, s_rcp, w[2 * g], w[2 * g + 1]);
-      sfword |= sb << (8 * g);
+      sb2 |= sb << (8 * g);
     }
-    if (m < M) {
-      uint4* dst = reinterpret_cast<uint4*>(Xq + (int64_t)m * (K >> 1) + c * 32);
-      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    }
-    if (m < Mpad) *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)m, (uint32_t)c, KS4)) = sfword;
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, sb2, 1);
+    if (m < M)
+      *reinterpret_cast<uint4*>(Xq + (int64_t)m * (K >> 1) + c * 32 + 8 * qg) = make_uint4(w[0], w[1], w[2], w[3]);
+    if ((lane & 1) == 0 && m < Mpad)
+      *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)m, (uint32_t)c, KS4)) = sb2 | (other << 16);
 
-    // ---- down-projection of the chunk on the tensor cores -----------------
+    // ---- down-projection of this warp's 16 rows on the tensor cores ---------
     if constexpr (R > 0) {
       const uint32_t sl_u32 = st_u32 + Cfg::kXBytes;
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        uint32_t a[2][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          const uint32_t arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          ldsm_x4(st_u32 + sw128(arow, ks * 2 + (lane >> 4)), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-        }
+        uint32_t a0, a1, a2, a3;
+        const uint32_t arow = 16 * half + (lane & 7) + ((lane >> 3) & 1) * 8;
+        ldsm_x4(st_u32 + sw128(arow, ks * 2 + (lane >> 4)), a0, a1, a2, a3);
 #pragma unroll
         for (int nt = 0; nt < Cfg::kNT; nt += 2) {
           uint32_t b[4];
-          if (nt + 1 < Cfg::kNT) {
-            const uint32_t brow = (nt + (lane >> 4)) * 8 + (lane & 7);
-            ldsm_x4(sl_u32 + sw128(brow, ks * 2 + ((lane >> 3) & 1)), b[0], b[1], b[2], b[3]);
-          } else {
-            const uint32_t brow = nt * 8 + (lane & 7);
-            ldsm_x2(sl_u32 + sw128(brow, ks * 2 + ((lane >> 3) & 1)), b[0], b[1]);
-            b[2] = b[3] = 0u;
-          }
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_bf16_16816(acc[mt * Cfg::kNT + nt], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b[0], b[1]);
-            if (nt + 1 < Cfg::kNT)
-              mma_bf16_16816(acc[mt * Cfg::kNT + nt + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b[2], b[3]);
-          }
+          const uint32_t brow = (nt + (lane >> 4)) * 8 + (lane & 7);
+          ldsm_x4(sl_u32 + sw128(brow, ks * 2 + ((lane >> 3) & 1)), b[0], b[1], b[2], b[3]);
+          mma_bf16_16816(acc[nt], a0, a1, a2, a3, b[0], b[1]);
+          mma_bf16_16816(acc[nt + 1], a0, a1, a2, a3, b[2], b[3]);
         }
       }
     }
@@ -238,23 +241,20 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
     if (lane == 0) mbar_arrive(&empty[s]);
   }
 
-  // ---- LAs = [hi | lo] of lr_scale * sum over warps of the partial X L1f ----
+  // ---- LAs = [hi | lo] of lr_scale * sum over pairs of the partial X L1f ----
   if constexpr (R > 0) {
     // Every chunk has been consumed, so no load is in flight into the ring: reuse it.
     named_bar_sync(1, QA_CONSUMER_WARPS * 32);
-    float* red = reinterpret_cast<float*>(smem);            // [warp][row][R]
+    float* red = reinterpret_cast<float*>(smem);            // [pair][row][R]
     if (ok) {
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < Cfg::kNT; ++nt) {
-          const int row = mt * 16 + (lane >> 2);
-          const int col = nt * 8 + 2 * (lane & 3);
-          float* p = red + ((warp * QA_ROWS + row) * R + col);
-          *reinterpret_cast<float2*>(p) = make_float2(acc[mt * Cfg::kNT + nt][0], acc[mt * Cfg::kNT + nt][1]);
-          *reinterpret_cast<float2*>(p + 8 * R) =
-              make_float2(acc[mt * Cfg::kNT + nt][2], acc[mt * Cfg::kNT + nt][3]);
-        }
+      for (int nt = 0; nt < Cfg::kNT; ++nt) {
+        const int row = 16 * half + (lane >> 2);
+        const int col = nt * 8 + 2 * (lane & 3);
+        float* p = red + ((pairi * QA_ROWS + row) * R + col);
+        *reinterpret_cast<float2*>(p) = make_float2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<float2*>(p + 8 * R) = make_float2(acc[nt][2], acc[nt][3]);
+      }
     }
     named_bar_sync(1, QA_CONSUMER_WARPS * 32);
     if (ok && !*abort_flag) {
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
         const int col = 2 * (p % (R / 2));
         float v0 = 0.0f, v1 = 0.0f;
 #pragma unroll
-        for (int w2 = 0; w2 < QA_CONSUMER_WARPS; ++w2) {
+        for (int w2 = 0; w2 < QA_PAIRS; ++w2) {
           const float2 t = *reinterpret_cast<const float2*>(red + ((w2 * QA_ROWS + row) * R + col));
           v0 += t.x;
           v1 += t.y;

@@ -86,20 +86,6 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Scale-factor buffer in MMA scale order viewed as 512-byte atoms: uint8 {256, 2, atoms},
-// box {256, 2, 4} = the 4 K-atoms (2 KB) of one 128-row block for one 256-wide K tile.
-bool make_map_sf(CUtensorMap* m, const void* base, uint64_t atoms) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {256, 2, atoms};
-  cuuint64_t strides[2] = {256, 512};
-  cuuint32_t box[3] = {256, 2, 4};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // ------------------------------------------------------------- checks -------
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -162,19 +148,17 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   DevInfo* d;
   if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
 
-  CUtensorMap tm_xq, tm_wq, tm_las, tm_l2p, tm_sfx, tm_sfw;
+  CUtensorMap tm_xq, tm_wq, tm_las, tm_l2p;
   if (!make_map_2d(&tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
-                   128) ||
+                   LN_BM) ||
       !make_map_2d(&tm_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128,
-                   128) ||
-      !make_map_sf(&tm_sfx, SFx, (uint64_t)(pad128(M) / 128) * (uint64_t)(K / 64)) ||
-      !make_map_sf(&tm_sfw, SFw, (uint64_t)(pad128(N) / 128) * (uint64_t)(K / 64)))
+                   LN_BN))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
     if (!make_map_2d(&tm_las, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, LAs, (uint64_t)2 * r, (uint64_t)M,
-                     (uint64_t)4 * r, 64, 128) ||
+                     (uint64_t)4 * r, 64, LN_BM) ||
         !make_map_2d(&tm_l2p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2p, (uint64_t)2 * r, (uint64_t)N,
-                     (uint64_t)4 * r, 64, 128))
+                     (uint64_t)4 * r, 64, LN_BN))
       return SVDQ_ERR_CUDA;
   } else {
     tm_las = tm_xq;
@@ -186,6 +170,8 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
     d->linear_attr = true;
   }
   LinearArgs a;
+  a.SFx = SFx;
+  a.SFw = SFw;
   a.bias = bias;
   a.Y = Y;
   a.y_fp32 = y_fp32;
@@ -197,9 +183,8 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   a.debug = debug;
   a.timeout_ns = timeout_ns ? timeout_ns : LN_DEFAULT_TIMEOUT_NS;
   const int64_t tiles = ((M + LN_BM - 1) / LN_BM) * ((N + LN_BN - 1) / LN_BN);
-  const int64_t pairs = tiles < d->sms / 2 ? tiles : d->sms / 2;
-  const int grid = (int)(2 * pairs);
-  k_linear<<<grid, LN_THREADS, LN_SMEM, s>>>(tm_xq, tm_wq, tm_las, tm_l2p, tm_sfx, tm_sfw, a);
+  const int grid = (int)(tiles < d->sms ? tiles : d->sms);
+  k_linear<<<grid, LN_THREADS, LN_SMEM, s>>>(tm_xq, tm_wq, tm_las, tm_l2p, a);
   return launch_status();
 }
 
