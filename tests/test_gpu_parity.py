@@ -173,3 +173,25 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert C.svdq_get_device_error()[0] == 0
     Y_or, _, _ = OL.svdq_reference(wl.X, dec.inv_s, dec.gs_x, dec.L1f, dec.L2b, dec.R32, wl.bias)
     check_y(Y2.float().cpu().numpy().astype(np.float64), Y_or, bf16=True)
+
+
+def test_repeated_launches_are_identical_and_error_free():
+    # Pipelines with many barriers in flight: repeat the forward and require bit-identical results
+    # and a clean device error word (catches ordering races that a single launch may miss).
+    M, K, N, r = 1152, 3072, 1536, 32
+    wl = small_case(M, K, N, r, seed=77)
+    dec = oracle_layer(wl, r)
+    g = GpuLayer(dec, wl.bias)
+    X = bf16_dev(wl.X)
+    ref = None
+    for _ in range(40):
+        Xq, SFx, LAs = g.quantize(X)
+        Y = g.linear(Xq, SFx, LAs)
+        torch.cuda.synchronize()
+        cur = (Xq.cpu().numpy().tobytes(), SFx.cpu().numpy().tobytes(), LAs.view(torch.int16).cpu().numpy().tobytes(),
+               Y.view(torch.int16).cpu().numpy().tobytes())
+        if ref is None:
+            ref = cur
+        else:
+            assert cur == ref
+    g.check_errors()
