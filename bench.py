@@ -68,6 +68,22 @@ def layer_flops(M, K, N, r):
     return 2.0 * M * N * K + 2.0 * M * r * (K + N)
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(flops_per_rank_step, world, ms_per_step_max):
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's step time (weak scaling)."""
+    return flops_per_rank_step * world / (ms_per_step_max * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------- clocks ------
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -266,10 +282,7 @@ def run_ours(args):
     ms = t_start.elapsed_time(t_end) / args.steps
     t_qa = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     t_ln = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
-    if world > 1:
-        t = torch.tensor([ms, t_qa, t_ln], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, t_qa, t_ln = [float(v) for v in t.tolist()]
+    ms, t_qa, t_ln = max_over_ranks([ms, t_qa, t_ln], device=dev)
 
     # end to end through the public API with host buffers (H2D of X, D2H of Y inside the timed region)
     Xh = X0.pin_memory()
@@ -287,14 +300,10 @@ def run_ours(args):
         layers[i % N_COPIES].forward_host(Xh, Yh, Xs[i % N_COPIES], Ys[i % N_COPIES])
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], device=dev)[0]
 
     fl = layer_flops(M, K, N, r)
-    value = fl * world / (ms * 1e-3) / 1e12
+    value = job_throughput(fl, world, ms)
     bf16_peak, hbm_peak, peak_kind = peaks()
     fp4_peak = bf16_peak * FP4_OVER_BF16
     lin_flops = 2.0 * M * N * K + 2.0 * M * N * r
@@ -317,7 +326,7 @@ def run_ours(args):
                                           "frac": qa_gbs / hbm_peak, "algorithmic_bytes": qa_bytes},
                     "svdq_linear": {"ms": t_ln, "TFLOP_per_s": lin_tf}},
         "clocks": clk,
-        "e2e": {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_throughput(fl, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 2), "ms_per_step": e2e_ms},
         "gpu_launches": 2 * args.steps,
     }
