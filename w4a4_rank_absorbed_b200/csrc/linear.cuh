@@ -19,9 +19,9 @@
 //            serviced one after another, so no lane has more than one in flight.
 //   warp 1   TMEM owner and MMA issuer (one thread): 4 MMAs (K = 64 each) per K tile,
 //            then the rank tiles, all into one accumulator.
-//   warp 2   scale copier (one thread): shared -> TMEM copies of each stage's scale blocks
-//            (tcgen05.cp, replicated into the four lane quarters), then a commit that tells
-//            the MMA thread the stage is ready.  Copies issued by the MMA thread itself
+//   warp 2   scale copier (one thread): as soon as a stage's scale blocks land (their own
+//            barrier, ahead of the larger A/B boxes), shared -> TMEM copies (tcgen05.cp,
+//            replicated into the four lane quarters), then a commit that tells the MMA thread.  Copies issued by the MMA thread itself
 //            stall its MMA issue; from a thread of their own they overlap the MMAs.
 //   warps 4-11  epilogue: TMEM -> registers (two warps per 32-lane quarter, 128 columns
 //            each), release the accumulator, scale + bias, store.
@@ -50,7 +50,7 @@ constexpr int LN_OFF_B = LN_STAGES * LN_A_BYTES;
 constexpr int LN_OFF_SFA = LN_OFF_B + LN_STAGES * LN_B_BYTES;
 constexpr int LN_OFF_SFB = LN_OFF_SFA + LN_STAGES * LN_SFA_BYTES;
 constexpr int LN_OFF_BAR = LN_OFF_SFB + LN_STAGES * LN_SFB_BYTES;
-constexpr int LN_SMEM = LN_OFF_BAR + 256 + 1024;
+constexpr int LN_SMEM = LN_OFF_BAR + 512 + 1024;
 constexpr uint64_t LN_DEFAULT_TIMEOUT_NS = 2000000000ull;
 static_assert(LN_SF_COL0 + LN_STAGES * LN_SF_COLS_PER_STAGE <= LN_TMEM_COLS, "TMEM budget");
 static_assert(LN_STAGES * LN_STREAMS <= 32, "one producer lane per slot and stream");
@@ -81,14 +81,15 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
   uint8_t* sB = smem + LN_OFF_B;
   uint8_t* sSFA = smem + LN_OFF_SFA;
   uint8_t* sSFB = smem + LN_OFF_SFB;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + LN_OFF_BAR);   // stage landed
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + LN_OFF_BAR);   // stage's A/B landed
   uint64_t* sf_ready = full + LN_STAGES;                              // stage scales in TMEM
   uint64_t* empty = sf_ready + LN_STAGES;                             // stage consumed by the MMAs
   uint64_t* acc_full = empty + LN_STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;                                    // MMA thread, on a time-out
   uint64_t* drain_cp = drain + 1;                                     // copier thread, on a time-out
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_cp + 1);
+  uint64_t* sf_full = drain_cp + 1;                                   // stage's scale blocks landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + LN_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
   if (threadIdx.x == 0) {
     for (int s = 0; s < LN_STAGES; ++s) {
       mbar_init(&full[s], 1);
+      mbar_init(&sf_full[s], 1);
       mbar_init(&sf_ready[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -157,19 +159,19 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
             const bool has_a = mb < sfx_blocks;
             const bool has_b0 = 2 * nb < sfw_blocks, has_b1 = 2 * nb + 1 < sfw_blocks;
             if (k == 0) {
-              mbar_arrive_expect_tx(&full[stage], (uint32_t)(LN_A_BYTES + LN_B_BYTES +
-                                                             (has_a + has_b0 + has_b1) * ka * 512));
+              mbar_arrive_expect_tx(&full[stage], (uint32_t)(LN_A_BYTES + LN_B_BYTES));
               tma_load_2d(sA + stage * LN_A_BYTES, &tm_xq, &full[stage], kt * 128, mb * LN_BM);
             } else if (k == 1) {
               tma_load_2d(sB + stage * LN_B_BYTES, &tm_wq, &full[stage], kt * 128, nb * LN_BN);
             } else if (k == 2) {
+              mbar_arrive_expect_tx(&sf_full[stage], (uint32_t)((has_a + has_b0 + has_b1) * ka * 512));
               if (has_a)
                 bulk_load(sSFA + stage * LN_SFA_BYTES, args.SFx + ((int64_t)mb * KA + 4 * kt) * 512,
-                          (uint32_t)(ka * 512), &full[stage]);
+                          (uint32_t)(ka * 512), &sf_full[stage]);
             } else if (k == 3 ? has_b0 : has_b1) {
               const int rb = 2 * nb + (k - 3);
               bulk_load(sSFB + stage * LN_SFB_BYTES + 2048 * (k - 3), args.SFw + ((int64_t)rb * KA + 4 * kt) * 512,
-                        (uint32_t)(ka * 512), &full[stage]);
+                        (uint32_t)(ka * 512), &sf_full[stage]);
             }
           } else {
             const int i = kt - nkt;
@@ -178,6 +180,8 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
               tma_load_2d(sA + stage * LN_A_BYTES, &tm_las, &full[stage], i * 64, mb * LN_BM);
             } else if (k == 1) {
               tma_load_2d(sB + stage * LN_B_BYTES, &tm_l2p, &full[stage], i * 64, nb * LN_BN);
+            } else if (k == 2) {
+              mbar_arrive(&sf_full[stage]);            // no scales in a rank stage
             }
           }
           issued = true;
@@ -187,7 +191,8 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
       if (*abort_flag && issued) {
         // Give the last load of this lane's slot the chance to land before the CTA exits.
         int never = 0;
-        mbar_wait(&full[g], last_parity, tmo, &never, 0x302);
+        if (k < 2) mbar_wait(&full[g], last_parity, tmo, &never, 0x302);
+        else mbar_wait(&sf_full[g], last_parity, tmo, &never, 0x302);
       }
     }
   } else if (warp == 1) {
@@ -203,8 +208,11 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
         if (it > 0 && !mbar_wait(acc_empty, (uint32_t)((it - 1) & 1), tmo, abort_flag, 0x311)) break;
         tc_fence_after();
         for (int kt = 0; kt < nst; ++kt) {
-          // sf_ready completes after the stage's data landed and its scales reached TMEM
-          if (!mbar_wait(&sf_ready[stage], phase, tmo, abort_flag, 0x312)) { ok = false; break; }
+          if (!mbar_wait(&full[stage], phase, tmo, abort_flag, 0x312) ||
+              !mbar_wait(&sf_ready[stage], phase, tmo, abort_flag, 0x314)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + stage * LN_A_BYTES));
           const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + stage * LN_B_BYTES));
@@ -239,8 +247,9 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         for (int kt = 0; kt < nst; ++kt) {
-          // the stage landed; the MMAs of the slot's previous round finished before its loads began
-          if (!mbar_wait(&full[stage], phase, tmo, abort_flag, 0x331)) { ok = false; break; }
+          // the stage's scales landed; the MMAs of the slot's previous round finished before its
+          // loads began, so its TMEM scale slot is free
+          if (!mbar_wait(&sf_full[stage], phase, tmo, abort_flag, 0x331)) { ok = false; break; }
           tc_fence_after();
           if (kt < nkt) {
             const int ka = min(4, KA - 4 * kt);

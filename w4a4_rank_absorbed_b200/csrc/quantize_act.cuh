@@ -13,8 +13,8 @@
 // The K axis is cut into 64-column chunks; chunk c goes through ring stage
 // c % S and is consumed by warp pair c % 7, so seven chunks are processed at
 // once and up to S loads are in flight (S = 14, or 7 for r > 88; S is a multiple of 7).  A stage holds the X box (32 x 64
-// bf16, 128-byte swizzle) and the L1f^T box (r x 64 bf16, same swizzle); the
-// 64 smoothing factors of the chunk are read through the read-only cache.  Warp h of a pair owns rows 16h..16h+15
+// bf16, 128-byte swizzle), the L1f^T box (r x 64 bf16, same swizzle) and the
+// chunk's 64 smoothing factors.  Warp h of a pair owns rows 16h..16h+15
 // of the chunk: two lanes per row quantize two groups of 16 each, and the
 // warp runs the 16 x r down-projection of its rows for the chunk's 64 columns
 // (mma.sync m16n8k16), keeping a partial sum in registers.  After the last
@@ -46,7 +46,8 @@ struct QaCfg {
   static constexpr int kRedBytes = QA_PAIRS * QA_ROWS * R * 4;
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kRedBytes <= kRingBytes, "reduction buffer must fit in the ring");
-  static constexpr int kRcpOff = kRingBytes;                        // 128-entry 1/d table
+  static constexpr int kInvOff = kRingBytes;                        // S x 64 smoothing factors
+  static constexpr int kRcpOff = kInvOff + kStages * 256;           // 128-entry 1/d table
   static constexpr int kBarOff = kRcpOff + 128 * 4;
   static constexpr int kSmem = kBarOff + 2 * kStages * 8 + 16 + 1024;
 };
@@ -76,36 +77,40 @@ SVDQ_DEV uint32_t sw128(uint32_t row, uint32_t c16) { return row * 128u + ((c16 
 
 // One group of 16 values of X (two 16-byte smem chunks) times 16 smoothing factors:
 // returns the UE4M3 scale and the two 32-bit code words.
+// d = a * b element-wise on two float32 pairs (two correctly rounded products).
+SVDQ_DEV float2 mul_f32x2(float2 a, float2 b) {
+  uint64_t d;
+  const uint64_t x = (uint64_t)__float_as_uint(a.x) | ((uint64_t)__float_as_uint(a.y) << 32);
+  const uint64_t y = (uint64_t)__float_as_uint(b.x) | ((uint64_t)__float_as_uint(b.y) << 32);
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(y));
+  return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
+}
+
+// One group of 16 values of X (two 16-byte smem chunks) times 16 smoothing factors:
+// returns the UE4M3 scale and the two 32-bit code words.
 SVDQ_DEV uint32_t quant_group(const uint4& r0, const uint4& r1, const float4* inv, float c_x,
                               const float* rcp_table, uint32_t& w0, uint32_t& w1) {
-  const float4 s0 = inv[0], s1 = inv[1], s2 = inv[2], s3 = inv[3];
-  float xh[16];
-  xh[0] = __fmul_rn(bf16_lo(r0.x), s0.x);
-  xh[1] = __fmul_rn(bf16_hi(r0.x), s0.y);
-  xh[2] = __fmul_rn(bf16_lo(r0.y), s0.z);
-  xh[3] = __fmul_rn(bf16_hi(r0.y), s0.w);
-  xh[4] = __fmul_rn(bf16_lo(r0.z), s1.x);
-  xh[5] = __fmul_rn(bf16_hi(r0.z), s1.y);
-  xh[6] = __fmul_rn(bf16_lo(r0.w), s1.z);
-  xh[7] = __fmul_rn(bf16_hi(r0.w), s1.w);
-  xh[8] = __fmul_rn(bf16_lo(r1.x), s2.x);
-  xh[9] = __fmul_rn(bf16_hi(r1.x), s2.y);
-  xh[10] = __fmul_rn(bf16_lo(r1.y), s2.z);
-  xh[11] = __fmul_rn(bf16_hi(r1.y), s2.w);
-  xh[12] = __fmul_rn(bf16_lo(r1.z), s3.x);
-  xh[13] = __fmul_rn(bf16_hi(r1.z), s3.y);
-  xh[14] = __fmul_rn(bf16_lo(r1.w), s3.z);
-  xh[15] = __fmul_rn(bf16_hi(r1.w), s3.w);
-  float a = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(xh[i]));
-  const uint32_t sb = cvt_ue4m3(__fmul_rn(a, c_x));
-  const float rinv = rcp_table[sb];           // f32(1 / f32(dec(sb) * gs)); entry 0 is 0
-  float q0[8], q1[8];
+  const uint32_t xw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+  float2 xh[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    q0[i] = __fmul_rn(xh[i], rinv);
-    q1[i] = __fmul_rn(xh[8 + i], rinv);
+    const float4 s4 = inv[i >> 1];
+    const float2 sp = (i & 1) ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
+    xh[i] = mul_f32x2(make_float2(bf16_lo(xw[i]), bf16_hi(xw[i])), sp);
+  }
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fmaxf(fabsf(xh[i].x), fabsf(xh[i].y)));
+  const uint32_t sb = cvt_ue4m3(__fmul_rn(a, c_x));
+  const float rinv = rcp_table[sb];           // f32(1 / f32(dec(sb) * gs)); entry 0 is 0
+  const float2 rr = make_float2(rinv, rinv);
+  float q0[8], q1[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 p0 = mul_f32x2(xh[i], rr);
+    const float2 p1 = mul_f32x2(xh[4 + i], rr);
+    q0[2 * i] = p0.x; q0[2 * i + 1] = p0.y;
+    q1[2 * i] = p1.x; q1[2 * i + 1] = p1.y;
   }
   // rinv = 0 for an all-zero scale: every product is +-0; the codes are forced to 0.
   w0 = sb ? cvt_e2m1x8(q0) : 0u;
@@ -123,6 +128,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* s_inv = reinterpret_cast<float*>(smem + Cfg::kInvOff);
   float* s_rcp = reinterpret_cast<float*>(smem + Cfg::kRcpOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
   uint64_t* empty = full + S;
@@ -151,21 +157,22 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   if (warp == QA_CONSUMER_WARPS) {
     // ---------------------------------------------------------- producer --
     // Lane 2g + k serves ring slot g (chunks c with c % S == g) and stream k (0: X box,
-    // 1: L1f^T box).  A thread's TMA copies are serviced one after another, so each lane
-    // keeps at most one copy in flight.
+    // 1: L1f^T box and the chunk's 64 smoothing factors).  A thread's TMA copies are
+    // serviced one after another, so each lane keeps at most two copies in flight.
     const int g = lane >> 1, k = lane & 1;
-    if (g < S && (k == 0 || R > 0)) {
+    if (g < S) {
       if (lane == 0) tma_prefetch_desc(&tm_x);
-      if (lane == 1) tma_prefetch_desc(&tm_l1);
+      if (lane == 1 && R > 0) tma_prefetch_desc(&tm_l1);
       for (int c = g; c < nchunks; c += S) {
         const uint32_t parity = (uint32_t)((c / S) & 1);
         if (!mbar_wait(&empty[g], parity ^ 1u, timeout_ns, abort_flag, 0x201)) break;
         uint8_t* st = smem + g * Cfg::kStageBytes;
         if (k == 0) {
-          mbar_arrive_expect_tx(&full[g], Cfg::kStageBytes);
+          mbar_arrive_expect_tx(&full[g], Cfg::kStageBytes + 256);
           tma_load_2d(st, &tm_x, &full[g], c * QA_CHUNK, m0);
         } else {
-          tma_load_2d(st + Cfg::kXBytes, &tm_l1, &full[g], c * QA_CHUNK, 0);
+          if (R > 0) tma_load_2d(st + Cfg::kXBytes, &tm_l1, &full[g], c * QA_CHUNK, 0);
+          bulk_load(s_inv + g * 64, inv_s + (int64_t)c * QA_CHUNK, 256, &full[g]);
         }
       }
     }
@@ -188,19 +195,13 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   bool ok = true;
   for (int c = pairi; c < nchunks; c += QA_PAIRS) {
     const int s = c % S;
-    // smoothing factors of this lane's two groups (read-only path; issued before the wait)
-    float4 inv[8];
-    {
-      const float4* src = reinterpret_cast<const float4*>(inv_s + (int64_t)c * QA_CHUNK + 16 * qg);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) inv[i] = __ldg(src + i);
-    }
     if (!mbar_wait(&full[s], (uint32_t)((c / S) & 1), timeout_ns, abort_flag, 0x202)) {
       ok = false;
       break;
     }
     const uint8_t* st = smem + s * Cfg::kStageBytes;
     const uint32_t st_u32 = smem_u32(st);
+    const float4* inv = reinterpret_cast<const float4*>(s_inv + s * 64 + 16 * qg);
 
     // ---- quantize two groups of row qrow ------------------------------------
     uint32_t w[4];
