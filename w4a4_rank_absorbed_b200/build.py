@@ -10,6 +10,7 @@ build needs no GPU and no libcuda.
 from __future__ import annotations
 
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -19,6 +20,10 @@ ROOT = os.path.dirname(PKG_DIR)
 SRC = os.path.join(PKG_DIR, "csrc", "svdq.cu")
 OUT = os.path.join(PKG_DIR, "libsvdq.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# k_linear moves registers between its warpgroups with setmaxnreg; the split adds up to
+# 512 threads x 128 registers, so the kernel must be launched with exactly 128 a thread
+# (fewer at launch and a warpgroup's setmaxnreg.inc would wait for registers forever).
+LINEAR_ENTRY_REGS = 128
 
 
 def nvcc_path() -> str:
@@ -45,16 +50,31 @@ def build(verbose: bool = False, force: bool = False) -> str:
     if not force and up_to_date():
         return OUT
     cmd = [nvcc_path(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "-o", OUT + ".tmp", SRC]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
+           "-Xcompiler", "-fvisibility=hidden", "-Xptxas=-v", "-o", OUT + ".tmp", SRC]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stdout.write(res.stdout + res.stderr)
+    regs = entry_registers(res.stdout + res.stderr, "k_linear")
+    if regs != LINEAR_ENTRY_REGS:
+        os.remove(OUT + ".tmp")
+        raise RuntimeError(f"k_linear compiled to {regs} registers per thread at entry, expected "
+                           f"{LINEAR_ENTRY_REGS}: its setmaxnreg split would not add up")
     os.replace(OUT + ".tmp", OUT)
     return OUT
+
+
+def entry_registers(ptxas_log: str, kernel: str) -> int | None:
+    """Registers per thread that ptxas reports for the entry function whose name holds `kernel`."""
+    lines = ptxas_log.splitlines()
+    for i, line in enumerate(lines):
+        if "Compiling entry function" in line and kernel in line:
+            for nxt in lines[i + 1:i + 6]:
+                m = re.search(r"Used (\d+) registers", nxt)
+                if m:
+                    return int(m.group(1))
+    return None
 
 
 if __name__ == "__main__":

@@ -11,20 +11,24 @@
 //   Y    = f32(gs_x gs_w) * acc + bias
 // LAs was pre-scaled by 1/(gs_x gs_w) in kernel 2, so a single scale serves both branches.
 //
-// Persistent, warp-specialised kernel, one CTA per SM, 128 x 256 output tiles:
-//   warp 0   TMA producer, one lane per (ring slot, load stream): A box 128 rows x 128 B,
-//            B box 256 rows x 128 B (128-byte swizzle), and the stage's scale blocks
-//            (SFA: 4 K-atoms of the 128 rows, SFB: 4 K-atoms of each of the two 128-row
-//            blocks; stored in MMA order, so plain bulk copies).  A thread's TMA copies are
-//            serviced one after another, so no lane has more than one in flight.
+// Persistent, warp-specialised kernel, one CTA of 16 warps per SM, 128 x 256 output tiles:
+//   warp 0   TMA producer for A (box 128 rows x 128 B, 128-byte swizzle) and the stage's
+//            scale blocks (SFA: 4 K-atoms of the 128 rows, SFB: 4 K-atoms of each of the two
+//            128-row blocks; stored in MMA order, so plain bulk copies).  One lane per
+//            (ring slot, stream): a thread's copies are serviced one after another.
 //   warp 1   TMEM owner and MMA issuer (one thread): 4 MMAs (K = 64 each) per K tile,
 //            then the rank tiles, all into one accumulator.
-//   warp 2   scale copier (one thread): as soon as a stage's scale blocks land (their own
-//            barrier, ahead of the larger A/B boxes), shared -> TMEM copies (tcgen05.cp,
-//            replicated into the four lane quarters), then a commit that tells the MMA thread.  Copies issued by the MMA thread itself
-//            stall its MMA issue; from a thread of their own they overlap the MMAs.
-//   warps 4-11  epilogue: TMEM -> registers (two warps per 32-lane quarter, 128 columns
-//            each), release the accumulator, scale + bias, store.
+//   warp 2   TMA producer for B (two boxes of 128 rows x 128 B).  The producers walk the
+//            stages in order with warp-uniform waits.
+//   warps 4-11   epilogue: TMEM -> registers (two warps per 32-lane quarter, 128 columns
+//            each), release the accumulator, scale + bias, 32-byte stores.
+//   warps 12-15  scale writers, one per TMEM lane quarter: shared -> registers ->
+//            tcgen05.st of the stage's 12 scale atoms into the quarter's lanes (the MMA
+//            reads each atom replicated in all four quarters).  Four warps storing in
+//            parallel take about a quarter of the time of the 12 tcgen05.cp copies a
+//            single thread would issue, which kept the MMAs waiting.
+// Registers: launched at 128 per thread; the epilogue warpgroups raise theirs to 168 and
+// the other two lower theirs to 88 (88 x 128 + 168 x 256 + 88 x 128 = 512 x 128).
 // 4-stage smem ring (54 KB a stage).  TMEM: accumulator in columns 0-255, per-stage
 // scale slots of 48 columns from column 256.
 #pragma once
@@ -37,23 +41,29 @@ constexpr int LN_BN = 256;
 constexpr int LN_STAGES = 4;
 constexpr int LN_A_BYTES = LN_BM * 128;          // 128 rows x 256 FP4 (or 64 bf16)
 constexpr int LN_B_BYTES = LN_BN * 128;
+constexpr int LN_B_HALF = LN_B_BYTES / 2;
 constexpr int LN_SFA_BYTES = 4 * 512;            // 4 K-atoms of 128 rows
 constexpr int LN_SFB_BYTES = 2 * 4 * 512;        // 2 row blocks x 4 K-atoms
-constexpr int LN_THREADS = 384;
+constexpr int LN_THREADS = 512;
 constexpr int LN_EPI_WARP0 = 4;
 constexpr int LN_EPI_WARPS = 8;
+constexpr int LN_SFW_WARP0 = 12;                 // scale writers: warps 12-15 (lane quarters 0-3)
 constexpr int LN_TMEM_COLS = 512;
 constexpr int LN_SF_COL0 = 256;
 constexpr int LN_SF_COLS_PER_STAGE = 48;
-constexpr int LN_STREAMS = 5;                    // A, B, SFA, SFB block 0, SFB block 1
+constexpr int LN_REGS_LOW = 88;                  // warpgroups 0 and 3
+constexpr int LN_REGS_HIGH = 168;                // warpgroups 1 and 2 (epilogue)
+constexpr int LN_A_STREAMS = 4;                  // warp 0 lanes per slot: A, SFA, SFB 0, SFB 1
+constexpr int LN_B_STREAMS = 2;                  // warp 2 lanes per slot: B rows 0-127, 128-255
 constexpr int LN_OFF_B = LN_STAGES * LN_A_BYTES;
 constexpr int LN_OFF_SFA = LN_OFF_B + LN_STAGES * LN_B_BYTES;
 constexpr int LN_OFF_SFB = LN_OFF_SFA + LN_STAGES * LN_SFA_BYTES;
 constexpr int LN_OFF_BAR = LN_OFF_SFB + LN_STAGES * LN_SFB_BYTES;
-constexpr int LN_SMEM = LN_OFF_BAR + 512 + 1024;
+constexpr int LN_SMEM = LN_OFF_BAR + 256 + 1024;
 constexpr uint64_t LN_DEFAULT_TIMEOUT_NS = 2000000000ull;
 static_assert(LN_SF_COL0 + LN_STAGES * LN_SF_COLS_PER_STAGE <= LN_TMEM_COLS, "TMEM budget");
-static_assert(LN_STAGES * LN_STREAMS <= 32, "one producer lane per slot and stream");
+static_assert(LN_STAGES * LN_A_STREAMS <= 32 && LN_STAGES * LN_B_STREAMS <= 32, "one lane per slot and stream");
+static_assert(LN_REGS_LOW * 256 + LN_REGS_HIGH * 256 == LN_THREADS * 128, "register split = launch budget");
 
 enum : int { LN_DBG_NO_LOADS = 1 };
 
@@ -63,6 +73,8 @@ struct LinearArgs {
   const uint16_t* bias;
   void* Y;
   int y_fp32;
+  int y_vec32;          // Y is 32-byte aligned: 32-byte stores
+
   int M, N, K, r;
   float gs;
   int debug;
@@ -71,9 +83,9 @@ struct LinearArgs {
 
 __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     const __grid_constant__ CUtensorMap tm_xq,   // uint8 {K/2, M},  box {128, 128}, SW128
-    const __grid_constant__ CUtensorMap tm_wq,   // uint8 {K/2, N},  box {128, 256}, SW128
+    const __grid_constant__ CUtensorMap tm_wq,   // uint8 {K/2, N},  box {128, 128}, SW128
     const __grid_constant__ CUtensorMap tm_las,  // bf16  {2r, M},   box {64, 128},  SW128
-    const __grid_constant__ CUtensorMap tm_l2p,  // bf16  {2r, N},   box {64, 256},  SW128
+    const __grid_constant__ CUtensorMap tm_l2p,  // bf16  {2r, N},   box {64, 128},  SW128
     const LinearArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -82,14 +94,13 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
   uint8_t* sSFA = smem + LN_OFF_SFA;
   uint8_t* sSFB = smem + LN_OFF_SFB;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + LN_OFF_BAR);   // stage's A/B landed
-  uint64_t* sf_ready = full + LN_STAGES;                              // stage scales in TMEM
+  uint64_t* sf_full = full + LN_STAGES;                               // stage's scale blocks landed
+  uint64_t* sf_ready = sf_full + LN_STAGES;                           // stage scales in TMEM
   uint64_t* empty = sf_ready + LN_STAGES;                             // stage consumed by the MMAs
   uint64_t* acc_full = empty + LN_STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;                                    // MMA thread, on a time-out
-  uint64_t* drain_cp = drain + 1;                                     // copier thread, on a time-out
-  uint64_t* sf_full = drain_cp + 1;                                   // stage's scale blocks landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + LN_STAGES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -110,13 +121,12 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     for (int s = 0; s < LN_STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&sf_full[s], 1);
-      mbar_init(&sf_ready[s], 1);
+      mbar_init(&sf_ready[s], 4);                  // one arrival per scale-writer warp
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, LN_EPI_WARPS);
     mbar_init(drain, 1);
-    mbar_init(drain_cp, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -129,16 +139,27 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane < LN_STAGES * LN_STREAMS && !(args.debug & LN_DBG_NO_LOADS)) {
-      // ---------------------------------------------------------- producer --
-      const int g = lane / LN_STREAMS, k = lane % LN_STREAMS;   // ring slot, load stream
+  // Register split by warpgroup: every warp of a warpgroup executes the same setmaxnreg, at
+  // the top of its role so that the role's code is compiled under that budget.
+  if (warp == 0 || warp == 2) {
+    regs_dec<LN_REGS_LOW>();
+    if (!(args.debug & LN_DBG_NO_LOADS)) {
+      // --------------------------------------------------------- producers --
+      // Both producer warps walk the stages in order with warp-uniform waits (lane 0 polls,
+      // the verdict is broadcast); each lane issues only its own (slot, stream) copy.
+      // Lanes that waited on different barriers in divergent branches would block one
+      // another inside try_wait.
+      const bool is_a = warp == 0;
+      const int per = is_a ? LN_A_STREAMS : LN_B_STREAMS;
+      const int g = lane / per, k = lane % per;    // ring slot, stream within the warp
+      const bool loader = lane < LN_STAGES * per;
       if (lane == 0) {
-        tma_prefetch_desc(&tm_xq);
-        tma_prefetch_desc(&tm_wq);
-        if (r > 0) {
-          tma_prefetch_desc(&tm_las);
-          tma_prefetch_desc(&tm_l2p);
+        if (is_a) {
+          tma_prefetch_desc(&tm_xq);
+          if (r > 0) tma_prefetch_desc(&tm_las);
+        } else {
+          tma_prefetch_desc(&tm_wq);
+          if (r > 0) tma_prefetch_desc(&tm_l2p);
         }
       }
       int gidx = 0;                 // position in this CTA's sequence of ring stages
@@ -148,55 +169,60 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
         const int mb = t / num_n, nb = t % num_n;
         for (int kt = 0; kt < nst; ++kt, ++gidx) {
           const int stage = gidx % LN_STAGES;
-          if (stage != g) continue;
           const uint32_t phase = (uint32_t)((gidx / LN_STAGES) & 1);
-          if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag, 0x301)) { ok = false; break; }
-          if (kt < nkt) {
-            // Scale blocks are contiguous runs of ka 512-byte atoms, copied as they are.  Blocks
-            // past the end of a scale buffer (rows beyond the padded M or N) are not loaded; they
-            // only feed accumulator rows or columns that are never stored.
-            const int ka = min(4, KA - 4 * kt);
-            const bool has_a = mb < sfx_blocks;
-            const bool has_b0 = 2 * nb < sfw_blocks, has_b1 = 2 * nb + 1 < sfw_blocks;
-            if (k == 0) {
-              mbar_arrive_expect_tx(&full[stage], (uint32_t)(LN_A_BYTES + LN_B_BYTES));
-              tma_load_2d(sA + stage * LN_A_BYTES, &tm_xq, &full[stage], kt * 128, mb * LN_BM);
-            } else if (k == 1) {
-              tma_load_2d(sB + stage * LN_B_BYTES, &tm_wq, &full[stage], kt * 128, nb * LN_BN);
-            } else if (k == 2) {
-              mbar_arrive_expect_tx(&sf_full[stage], (uint32_t)((has_a + has_b0 + has_b1) * ka * 512));
-              if (has_a)
-                bulk_load(sSFA + stage * LN_SFA_BYTES, args.SFx + ((int64_t)mb * KA + 4 * kt) * 512,
-                          (uint32_t)(ka * 512), &sf_full[stage]);
-            } else if (k == 3 ? has_b0 : has_b1) {
-              const int rb = 2 * nb + (k - 3);
-              bulk_load(sSFB + stage * LN_SFB_BYTES + 2048 * (k - 3), args.SFw + ((int64_t)rb * KA + 4 * kt) * 512,
-                        (uint32_t)(ka * 512), &sf_full[stage]);
-            }
-          } else {
+          int free_slot = 1;
+          if (lane == 0) free_slot = mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag, 0x301) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, free_slot, 0)) { ok = false; break; }
+          if (loader && g == stage) {
+            const bool lr = kt >= nkt;             // a rank stage: LAs x L2p in bf16
             const int i = kt - nkt;
-            if (k == 0) {
-              mbar_arrive_expect_tx(&full[stage], LN_A_BYTES + LN_B_BYTES);
-              tma_load_2d(sA + stage * LN_A_BYTES, &tm_las, &full[stage], i * 64, mb * LN_BM);
-            } else if (k == 1) {
-              tma_load_2d(sB + stage * LN_B_BYTES, &tm_l2p, &full[stage], i * 64, nb * LN_BN);
-            } else if (k == 2) {
-              mbar_arrive(&sf_full[stage]);            // no scales in a rank stage
+            if (is_a) {
+              if (k == 0) {
+                mbar_arrive_expect_tx(&full[stage], (uint32_t)(LN_A_BYTES + LN_B_BYTES));
+                if (lr) tma_load_2d(sA + stage * LN_A_BYTES, &tm_las, &full[stage], i * 64, mb * LN_BM);
+                else tma_load_2d(sA + stage * LN_A_BYTES, &tm_xq, &full[stage], kt * 128, mb * LN_BM);
+              } else if (lr) {
+                if (k == 1) mbar_arrive(&sf_full[stage]);   // no scales in a rank stage
+              } else {
+                // Scale blocks are contiguous runs of ka 512-byte atoms, copied as they are.
+                // Blocks past the end of a scale buffer (rows beyond the padded M or N) are
+                // not loaded; they only feed accumulator rows or columns never stored.
+                const int ka = min(4, KA - 4 * kt);
+                const bool has_a = mb < sfx_blocks;
+                const bool has_b0 = 2 * nb < sfw_blocks, has_b1 = 2 * nb + 1 < sfw_blocks;
+                if (k == 1) {
+                  mbar_arrive_expect_tx(&sf_full[stage], (uint32_t)((has_a + has_b0 + has_b1) * ka * 512));
+                  if (has_a)
+                    bulk_load(sSFA + stage * LN_SFA_BYTES, args.SFx + ((int64_t)mb * KA + 4 * kt) * 512,
+                              (uint32_t)(ka * 512), &sf_full[stage]);
+                } else if (k == 2 ? has_b0 : has_b1) {
+                  const int hb = k - 2;
+                  bulk_load(sSFB + stage * LN_SFB_BYTES + 2048 * hb,
+                            args.SFw + ((int64_t)(2 * nb + hb) * KA + 4 * kt) * 512, (uint32_t)(ka * 512),
+                            &sf_full[stage]);
+                }
+              }
+            } else {
+              uint8_t* dst = sB + stage * LN_B_BYTES + k * LN_B_HALF;
+              if (lr) tma_load_2d(dst, &tm_l2p, &full[stage], i * 64, nb * LN_BN + k * 128);
+              else tma_load_2d(dst, &tm_wq, &full[stage], kt * 128, nb * LN_BN + k * 128);
             }
+            issued = true;
+            last_parity = phase;
           }
-          issued = true;
-          last_parity = phase;
+          __syncwarp();
         }
       }
       if (*abort_flag && issued) {
         // Give the last load of this lane's slot the chance to land before the CTA exits.
         int never = 0;
-        if (k < 2) mbar_wait(&full[g], last_parity, tmo, &never, 0x302);
-        else mbar_wait(&sf_full[g], last_parity, tmo, &never, 0x302);
+        if (is_a && k > 0) mbar_wait(&sf_full[g], last_parity, tmo, &never, 0x302);
+        else mbar_wait(&full[g], last_parity, tmo, &never, 0x302);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer --
+    regs_dec<LN_REGS_LOW>();
     if (lane == 0) {
       constexpr uint32_t IDESC_F4 = idesc_nvf4(LN_BM, LN_BN);
       constexpr uint32_t IDESC_BF16 = idesc_bf16(LN_BM, LN_BN);
@@ -239,42 +265,55 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
         mbar_wait(drain, 0, tmo, &never, 0x313);
       }
     }
-  } else if (warp == 2) {
-    // --------------------------------------------------------- scale copier --
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        for (int kt = 0; kt < nst; ++kt) {
-          // the stage's scales landed; the MMAs of the slot's previous round finished before its
-          // loads began, so its TMEM scale slot is free
-          if (!mbar_wait(&sf_full[stage], phase, tmo, abort_flag, 0x331)) { ok = false; break; }
-          tc_fence_after();
-          if (kt < nkt) {
-            const int ka = min(4, KA - 4 * kt);
-            const uint32_t sfa_col = tbase + LN_SF_COL0 + LN_SF_COLS_PER_STAGE * stage;
-            const uint32_t sfb_col = sfa_col + 16;
-            const uint32_t sfa_s = smem_u32(sSFA + stage * LN_SFA_BYTES);
-            const uint32_t sfb_s = smem_u32(sSFB + stage * LN_SFB_BYTES);
-            for (int j = 0; j < ka; ++j) {
-              tc_cp_32x128b_x4(sfa_col + 4 * j, sdesc_sf_block(sfa_s + 512 * j));
-              tc_cp_32x128b_x4(sfb_col + 8 * j, sdesc_sf_block(sfb_s + 512 * j));
-              tc_cp_32x128b_x4(sfb_col + 8 * j + 4, sdesc_sf_block(sfb_s + 2048 + 512 * j));
-            }
+  } else if (warp >= LN_SFW_WARP0) {
+    // -------------------------------------------------------- scale writers --
+    // Warp w writes TMEM lanes 32 (w % 4) .. +31.  Atom j of a 128-row scale block holds
+    // row r's 4 scales at byte 16 (r % 32) + 4 ((r / 32) % 4); lane l of every quarter
+    // takes the atom's 16 bytes at 16 l into 4 consecutive columns (the replicated layout
+    // the block-scaled MMA reads).  SFA atom j -> columns 4j, SFB block b atom j -> 16 + 8j + 4b.
+    regs_dec<LN_REGS_LOW>();
+    const int q = warp & 3;
+    const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int kt = 0; kt < nst; ++kt) {
+        // The stage's scales landed; the MMAs of the slot's previous round finished before its
+        // loads began, so the slot's TMEM columns are free.
+        int landed = 1;
+        if (lane == 0) landed = mbar_wait(&sf_full[stage], phase, tmo, abort_flag, 0x331) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, landed, 0)) { ok = false; break; }
+        if (kt < nkt) {
+          const uint8_t* sa = sSFA + stage * LN_SFA_BYTES + 16 * lane;
+          const uint8_t* sb = sSFB + stage * LN_SFB_BYTES + 16 * lane;
+          uint32_t a[16], b0[16], b1[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 x = *reinterpret_cast<const uint4*>(sa + 512 * j);
+            const uint4 y0 = *reinterpret_cast<const uint4*>(sb + 512 * j);
+            const uint4 y1 = *reinterpret_cast<const uint4*>(sb + 2048 + 512 * j);
+            a[4 * j] = x.x; a[4 * j + 1] = x.y; a[4 * j + 2] = x.z; a[4 * j + 3] = x.w;
+            uint32_t* b = j < 2 ? b0 : b1;
+            const int o = 8 * (j & 1);
+            b[o] = y0.x; b[o + 1] = y0.y; b[o + 2] = y0.z; b[o + 3] = y0.w;
+            b[o + 4] = y1.x; b[o + 5] = y1.y; b[o + 6] = y1.z; b[o + 7] = y1.w;
           }
-          tc_commit(&sf_ready[stage]);
-          if (++stage == LN_STAGES) { stage = 0; phase ^= 1u; }
+          const uint32_t col = lane_base + LN_SF_COL0 + LN_SF_COLS_PER_STAGE * stage;
+          tmem_st_32x32b_x16(col, a);
+          tmem_st_32x32b_x16(col + 16, b0);
+          tmem_st_32x32b_x16(col + 32, b1);
+          tmem_st_wait();
         }
-      }
-      if (*abort_flag) {
-        int never = 0;
-        tc_commit(drain_cp);     // lets the copies issued so far finish before TMEM is released
-        mbar_wait(drain_cp, 0, tmo, &never, 0x332);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_ready[stage]);
+        if (++stage == LN_STAGES) { stage = 0; phase ^= 1u; }
       }
     }
   } else if (warp >= LN_EPI_WARP0) {
     // ------------------------------------------------------------- epilogue --
+    regs_inc<LN_REGS_HIGH>();
     const int ew = warp - LN_EPI_WARP0;
     const int q = warp & 3;              // TMEM lane quarter this warp may access
     const int h = ew >> 2;               // column half of the 256-wide tile
@@ -297,41 +336,62 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
 
       const int row = mb * LN_BM + 32 * q + lane;
       if (row < M) {
+        // 16 columns at a time: one 32-byte store of bf16 (two of fp32); N % 16 == 0, so a
+        // group is either wholly inside the matrix or wholly past its end.
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int n = nb * LN_BN + h * 128 + 32 * i + 8 * g;
+          for (int gp = 0; gp < 2; ++gp) {
+            const int n = nb * LN_BN + h * 128 + 32 * i + 16 * gp;
             if (n < N) {
-              float bv[8];
+              float y[16];
               if (args.bias) {
-                const uint4 bw = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
-                bv[0] = bf16_lo(bw.x); bv[1] = bf16_hi(bw.x); bv[2] = bf16_lo(bw.y); bv[3] = bf16_hi(bw.y);
-                bv[4] = bf16_lo(bw.z); bv[5] = bf16_hi(bw.z); bv[6] = bf16_lo(bw.w); bv[7] = bf16_hi(bw.w);
+                const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
+                const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(args.bias + n + 8));
+                const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  y[2 * e] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 2 * e]), bf16_lo(bw[e]));
+                  y[2 * e + 1] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 2 * e + 1]), bf16_hi(bw[e]));
+                }
               } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) bv[e] = 0.0f;
+                for (int e = 0; e < 16; ++e) y[e] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + e]), 0.0f);
               }
-              float y[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) y[e] = __fmaf_rn(gs, __uint_as_float(v[i][8 * g + e]), bv[e]);
               if (args.y_fp32) {
-                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.Y) + (int64_t)row * N + n);
-                dst[0] = make_float4(y[0], y[1], y[2], y[3]);
-                dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+                float* dst = static_cast<float*>(args.Y) + (int64_t)row * N + n;
+                if (args.y_vec32) {
+                  st_global_v8(dst, __float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                               __float_as_uint(y[3]), __float_as_uint(y[4]), __float_as_uint(y[5]),
+                               __float_as_uint(y[6]), __float_as_uint(y[7]));
+                  st_global_v8(dst + 8, __float_as_uint(y[8]), __float_as_uint(y[9]), __float_as_uint(y[10]),
+                               __float_as_uint(y[11]), __float_as_uint(y[12]), __float_as_uint(y[13]),
+                               __float_as_uint(y[14]), __float_as_uint(y[15]));
+                } else {
+                  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) d4[e] = make_float4(y[4 * e], y[4 * e + 1], y[4 * e + 2], y[4 * e + 3]);
+                }
               } else {
-                uint4 o;
-                o.x = pack_bf16x2(y[0], y[1]);
-                o.y = pack_bf16x2(y[2], y[3]);
-                o.z = pack_bf16x2(y[4], y[5]);
-                o.w = pack_bf16x2(y[6], y[7]);
-                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.Y) + (int64_t)row * N + n) = o;
+                uint32_t o[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+                uint16_t* dst = static_cast<uint16_t*>(args.Y) + (int64_t)row * N + n;
+                if (args.y_vec32) {
+                  st_global_v8(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+                } else {
+                  uint4* d4 = reinterpret_cast<uint4*>(dst);
+                  d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                  d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                }
               }
             }
           }
         }
       }
     }
+  } else {
+    regs_dec<LN_REGS_LOW>();                       // warp 3: no role
   }
 
   tc_fence_before();

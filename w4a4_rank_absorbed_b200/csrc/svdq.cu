@@ -152,13 +152,13 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   if (!make_map_2d(&tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
                    LN_BM) ||
       !make_map_2d(&tm_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128,
-                   LN_BN))
+                   LN_BN / 2))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
     if (!make_map_2d(&tm_las, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, LAs, (uint64_t)2 * r, (uint64_t)M,
                      (uint64_t)4 * r, 64, LN_BM) ||
         !make_map_2d(&tm_l2p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2p, (uint64_t)2 * r, (uint64_t)N,
-                     (uint64_t)4 * r, 64, LN_BN))
+                     (uint64_t)4 * r, 64, LN_BN / 2))
       return SVDQ_ERR_CUDA;
   } else {
     tm_las = tm_xq;
@@ -175,6 +175,7 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   a.bias = bias;
   a.Y = Y;
   a.y_fp32 = y_fp32;
+  a.y_vec32 = (reinterpret_cast<uintptr_t>(Y) & 31u) == 0 ? 1 : 0;
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
