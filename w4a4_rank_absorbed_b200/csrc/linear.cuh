@@ -12,14 +12,13 @@
 // LAs was pre-scaled by 1/(gs_x gs_w) in kernel 2, so a single scale serves both branches.
 //
 // Persistent, warp-specialised kernel, one CTA of 16 warps per SM, 128 x 256 output tiles:
-//   warp 0   TMA producer for A (box 128 rows x 128 B, 128-byte swizzle) and the stage's
-//            scale blocks (SFA: 4 K-atoms of the 128 rows, SFB: 4 K-atoms of each of the two
-//            128-row blocks; stored in MMA order, so plain bulk copies).  One lane per
-//            (ring slot, stream): a thread's copies are serviced one after another.
+//   warp 0   TMA producer for A (box 128 rows x 128 B, 128-byte swizzle) and B (two boxes
+//            of 128 rows x 128 B), issued by three lanes in one converged instruction.
 //   warp 1   TMEM owner and MMA issuer (one thread): 4 MMAs (K = 64 each) per K tile,
 //            then the rank tiles, all into one accumulator.
-//   warp 2   TMA producer for B (two boxes of 128 rows x 128 B).  The producers walk the
-//            stages in order with warp-uniform waits.
+//   warp 2   producer for the stage's scale blocks (SFA: 4 K-atoms of the 128 rows, SFB:
+//            4 K-atoms of each of the two 128-row blocks; stored in MMA order, so plain
+//            bulk copies), again three lanes in one instruction.
 //   warps 4-11   epilogue: TMEM -> registers (two warps per 32-lane quarter, 128 columns
 //            each), release the accumulator, scale + bias, 32-byte stores.
 //   warps 12-15  scale writers, one per TMEM lane quarter: shared -> registers ->
@@ -53,8 +52,7 @@ constexpr int LN_SF_COL0 = 256;
 constexpr int LN_SF_COLS_PER_STAGE = 48;
 constexpr int LN_REGS_LOW = 88;                  // warpgroups 0 and 3
 constexpr int LN_REGS_HIGH = 168;                // warpgroups 1 and 2 (epilogue)
-constexpr int LN_A_STREAMS = 4;                  // warp 0 lanes per slot: A, SFA, SFB 0, SFB 1
-constexpr int LN_B_STREAMS = 2;                  // warp 2 lanes per slot: B rows 0-127, 128-255
+constexpr int LN_STREAMS = 3;                    // lanes per slot: A, B 0, B 1 (warp 0); SFA, SFB 0, SFB 1 (warp 2)
 constexpr int LN_OFF_B = LN_STAGES * LN_A_BYTES;
 constexpr int LN_OFF_SFA = LN_OFF_B + LN_STAGES * LN_B_BYTES;
 constexpr int LN_OFF_SFB = LN_OFF_SFA + LN_STAGES * LN_SFA_BYTES;
@@ -62,7 +60,7 @@ constexpr int LN_OFF_BAR = LN_OFF_SFB + LN_STAGES * LN_SFB_BYTES;
 constexpr int LN_SMEM = LN_OFF_BAR + 256 + 1024;
 constexpr uint64_t LN_DEFAULT_TIMEOUT_NS = 2000000000ull;
 static_assert(LN_SF_COL0 + LN_STAGES * LN_SF_COLS_PER_STAGE <= LN_TMEM_COLS, "TMEM budget");
-static_assert(LN_STAGES * LN_A_STREAMS <= 32 && LN_STAGES * LN_B_STREAMS <= 32, "one lane per slot and stream");
+static_assert(LN_STAGES * LN_STREAMS <= 32 && LN_STREAMS == 3, "one lane per slot and stream");
 static_assert(LN_REGS_LOW * 256 + LN_REGS_HIGH * 256 == LN_THREADS * 128, "register split = launch budget");
 
 enum : int { LN_DBG_NO_LOADS = 1 };
@@ -145,21 +143,27 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     regs_dec<LN_REGS_LOW>();
     if (!(args.debug & LN_DBG_NO_LOADS)) {
       // --------------------------------------------------------- producers --
-      // Both producer warps walk the stages in order with warp-uniform waits (lane 0 polls,
-      // the verdict is broadcast); each lane issues only its own (slot, stream) copy.
-      // Lanes that waited on different barriers in divergent branches would block one
-      // another inside try_wait.
-      const bool is_a = warp == 0;
-      const int per = is_a ? LN_A_STREAMS : LN_B_STREAMS;
-      const int g = lane / per, k = lane % per;    // ring slot, stream within the warp
-      const bool loader = lane < LN_STAGES * per;
+      // Warp 0 issues the stage's three tensor boxes (A; B rows 0-127; B rows 128-255),
+      // warp 2 its three scale blocks (SFA; SFB 0; SFB 1).  Lane 3g + k serves stream k of
+      // ring slot g, so no lane has two copies of the same stream in flight (a thread's
+      // copies are serviced one after another).  The three lanes of a stage issue one
+      // converged copy instruction with per-lane operands: an issuing warp is held for
+      // about the same time by a copy instruction whether one lane or three take part,
+      // so three lanes in divergent branches would take three times as long.  Both warps
+      // walk the stages in order with warp-uniform waits (lane 0 polls, the verdict is
+      // broadcast); lanes waiting on different barriers in divergent branches would block
+      // one another inside try_wait.
+      const bool tensor_warp = warp == 0;
+      const int g = lane / LN_STREAMS, k = lane % LN_STREAMS;   // ring slot, stream
+      const bool loader = lane < LN_STAGES * LN_STREAMS;
       if (lane == 0) {
-        if (is_a) {
+        if (tensor_warp) {
           tma_prefetch_desc(&tm_xq);
-          if (r > 0) tma_prefetch_desc(&tm_las);
-        } else {
           tma_prefetch_desc(&tm_wq);
-          if (r > 0) tma_prefetch_desc(&tm_l2p);
+          if (r > 0) {
+            tma_prefetch_desc(&tm_las);
+            tma_prefetch_desc(&tm_l2p);
+          }
         }
       }
       int gidx = 0;                 // position in this CTA's sequence of ring stages
@@ -173,42 +177,41 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
           int free_slot = 1;
           if (lane == 0) free_slot = mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag, 0x301) ? 1 : 0;
           if (!__shfl_sync(0xffffffffu, free_slot, 0)) { ok = false; break; }
-          if (loader && g == stage) {
-            const bool lr = kt >= nkt;             // a rank stage: LAs x L2p in bf16
-            const int i = kt - nkt;
-            if (is_a) {
-              if (k == 0) {
-                mbar_arrive_expect_tx(&full[stage], (uint32_t)(LN_A_BYTES + LN_B_BYTES));
-                if (lr) tma_load_2d(sA + stage * LN_A_BYTES, &tm_las, &full[stage], i * 64, mb * LN_BM);
-                else tma_load_2d(sA + stage * LN_A_BYTES, &tm_xq, &full[stage], kt * 128, mb * LN_BM);
-              } else if (lr) {
-                if (k == 1) mbar_arrive(&sf_full[stage]);   // no scales in a rank stage
-              } else {
-                // Scale blocks are contiguous runs of ka 512-byte atoms, copied as they are.
-                // Blocks past the end of a scale buffer (rows beyond the padded M or N) are
-                // not loaded; they only feed accumulator rows or columns never stored.
-                const int ka = min(4, KA - 4 * kt);
-                const bool has_a = mb < sfx_blocks;
-                const bool has_b0 = 2 * nb < sfw_blocks, has_b1 = 2 * nb + 1 < sfw_blocks;
-                if (k == 1) {
-                  mbar_arrive_expect_tx(&sf_full[stage], (uint32_t)((has_a + has_b0 + has_b1) * ka * 512));
-                  if (has_a)
-                    bulk_load(sSFA + stage * LN_SFA_BYTES, args.SFx + ((int64_t)mb * KA + 4 * kt) * 512,
-                              (uint32_t)(ka * 512), &sf_full[stage]);
-                } else if (k == 2 ? has_b0 : has_b1) {
-                  const int hb = k - 2;
-                  bulk_load(sSFB + stage * LN_SFB_BYTES + 2048 * hb,
-                            args.SFw + ((int64_t)(2 * nb + hb) * KA + 4 * kt) * 512, (uint32_t)(ka * 512),
-                            &sf_full[stage]);
-                }
-              }
-            } else {
-              uint8_t* dst = sB + stage * LN_B_BYTES + k * LN_B_HALF;
-              if (lr) tma_load_2d(dst, &tm_l2p, &full[stage], i * 64, nb * LN_BN + k * 128);
-              else tma_load_2d(dst, &tm_wq, &full[stage], kt * 128, nb * LN_BN + k * 128);
+          const bool mine = loader && g == stage;
+          const unsigned smask = 7u << (LN_STREAMS * stage);   // the stage's three lanes
+          const bool lr = kt >= nkt;               // a rank stage: LAs x L2p in bf16
+          if (tensor_warp) {
+            if (mine) {
+              if (k == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(LN_A_BYTES + LN_B_BYTES));
+              const CUtensorMap* map = k == 0 ? (lr ? &tm_las : &tm_xq) : (lr ? &tm_l2p : &tm_wq);
+              uint8_t* dst = k == 0 ? sA + stage * LN_A_BYTES : sB + stage * LN_B_BYTES + (k - 1) * LN_B_HALF;
+              const int x = lr ? (kt - nkt) * 64 : kt * 128;
+              const int y = k == 0 ? mb * LN_BM : nb * LN_BN + (k - 1) * 128;
+              __syncwarp(smask);
+              tma_load_2d(dst, map, &full[stage], x, y);
+              issued = true;
+              last_parity = phase;
             }
-            issued = true;
-            last_parity = phase;
+          } else if (mine) {
+            // Scale blocks are contiguous runs of ka 512-byte atoms, copied as they are.
+            // Blocks past the end of a scale buffer (rows beyond the padded M or N) are not
+            // loaded; they only feed accumulator rows or columns that are never stored.
+            const int ka = lr ? 0 : min(4, KA - 4 * kt);
+            const int has_a = mb < sfx_blocks, has_b0 = 2 * nb < sfw_blocks, has_b1 = 2 * nb + 1 < sfw_blocks;
+            if (k == 0) {
+              if (lr) mbar_arrive(&sf_full[stage]);        // no scales in a rank stage
+              else mbar_arrive_expect_tx(&sf_full[stage], (uint32_t)((has_a + has_b0 + has_b1) * ka * 512));
+            }
+            const bool has = !lr && (k == 0 ? has_a : k == 1 ? has_b0 : has_b1);
+            __syncwarp(smask);
+            if (has) {
+              uint8_t* dst = k == 0 ? sSFA + stage * LN_SFA_BYTES : sSFB + stage * LN_SFB_BYTES + 2048 * (k - 1);
+              const uint8_t* src = k == 0 ? args.SFx + ((int64_t)mb * KA + 4 * kt) * 512
+                                          : args.SFw + ((int64_t)(2 * nb + k - 1) * KA + 4 * kt) * 512;
+              bulk_load(dst, src, (uint32_t)(ka * 512), &sf_full[stage]);
+              issued = true;
+              last_parity = phase;
+            }
           }
           __syncwarp();
         }
@@ -216,8 +219,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
       if (*abort_flag && issued) {
         // Give the last load of this lane's slot the chance to land before the CTA exits.
         int never = 0;
-        if (is_a && k > 0) mbar_wait(&sf_full[g], last_parity, tmo, &never, 0x302);
-        else mbar_wait(&full[g], last_parity, tmo, &never, 0x302);
+        mbar_wait(tensor_warp ? &full[g] : &sf_full[g], last_parity, tmo, &never, 0x302);
       }
     }
   } else if (warp == 1) {
