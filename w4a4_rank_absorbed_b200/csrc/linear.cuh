@@ -65,6 +65,20 @@ static_assert(LN_REGS_LOW * 256 + LN_REGS_HIGH * 256 == LN_THREADS * 128, "regis
 
 enum : int { LN_DBG_NO_LOADS = 1 };
 
+#ifndef LN_RASTER_GM
+#define LN_RASTER_GM 12
+#endif
+// Output tile t -> (row block mb, column block nb).  Tiles run in groups of LN_RASTER_GM
+// row blocks; within a group the row block varies fastest.
+SVDQ_DEV void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
+  const int per_group = LN_RASTER_GM * num_n;
+  const int first_m = (t / per_group) * LN_RASTER_GM;
+  const int gm = min(LN_RASTER_GM, num_m - first_m);
+  const int w = t - (t / per_group) * per_group;
+  mb = first_m + w % gm;
+  nb = w / gm;
+}
+
 struct LinearArgs {
   const uint8_t* SFx;
   const uint8_t* SFw;
@@ -170,7 +184,8 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
       bool ok = true, issued = false;
       uint32_t last_parity = 0;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const int mb = t / num_n, nb = t % num_n;
+        int mb, nb;
+        tile_coords(t, num_m, num_n, mb, nb);
         for (int kt = 0; kt < nst; ++kt, ++gidx) {
           const int stage = gidx % LN_STAGES;
           const uint32_t phase = (uint32_t)((gidx / LN_STAGES) & 1);
@@ -322,7 +337,8 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     const float gs = args.gs;
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const int mb = t / num_n, nb = t % num_n;
+      int mb, nb;
+      tile_coords(t, num_m, num_n, mb, nb);
       if (!mbar_wait(acc_full, (uint32_t)(it & 1), tmo, abort_flag, 0x321)) break;
       tc_fence_after();
       uint32_t v[4][32];
