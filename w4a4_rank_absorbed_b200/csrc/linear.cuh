@@ -302,14 +302,14 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
         if (lane == 0) landed = mbar_wait(&sf_full[stage], phase, tmo, abort_flag, 0x331) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, landed, 0)) { ok = false; break; }
         if (kt < nkt) {
-          const uint8_t* sa = sSFA + stage * LN_SFA_BYTES + 16 * lane;
-          const uint8_t* sb = sSFB + stage * LN_SFB_BYTES + 16 * lane;
+          const uint32_t sa = smem_u32(sSFA + stage * LN_SFA_BYTES) + 16 * lane;
+          const uint32_t sb = smem_u32(sSFB + stage * LN_SFB_BYTES) + 16 * lane;
           uint32_t a[16], b0[16], b1[16];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint4 x = *reinterpret_cast<const uint4*>(sa + 512 * j);
-            const uint4 y0 = *reinterpret_cast<const uint4*>(sb + 512 * j);
-            const uint4 y1 = *reinterpret_cast<const uint4*>(sb + 2048 + 512 * j);
+            const uint4 x = lds_v4(sa + 512 * j);
+            const uint4 y0 = lds_v4(sb + 512 * j);
+            const uint4 y1 = lds_v4(sb + 2048 + 512 * j);
             a[4 * j] = x.x; a[4 * j + 1] = x.y; a[4 * j + 2] = x.z; a[4 * j + 3] = x.w;
             uint32_t* b = j < 2 ? b0 : b1;
             const int o = 8 * (j & 1);

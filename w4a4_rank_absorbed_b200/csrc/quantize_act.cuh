@@ -88,8 +88,8 @@ SVDQ_DEV float2 mul_f32x2(float2 a, float2 b) {
 
 // One group of 16 values of X (two 16-byte smem chunks) times 16 smoothing factors:
 // returns the UE4M3 scale and the two 32-bit code words.
-SVDQ_DEV uint32_t quant_group(const uint4& r0, const uint4& r1, const float4* inv, float c_x,
-                              const float* rcp_table, uint32_t& w0, uint32_t& w1) {
+SVDQ_DEV uint32_t quant_group(const uint4& r0, const uint4& r1, const float4 (&inv)[4], float c_x,
+                              uint32_t rcp_table, uint32_t& w0, uint32_t& w1) {
   const uint32_t xw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
   float2 xh[8];
 #pragma unroll
@@ -102,7 +102,7 @@ SVDQ_DEV uint32_t quant_group(const uint4& r0, const uint4& r1, const float4* in
 #pragma unroll
   for (int i = 0; i < 8; ++i) a = fmaxf(a, fmaxf(fabsf(xh[i].x), fabsf(xh[i].y)));
   const uint32_t sb = cvt_ue4m3(__fmul_rn(a, c_x));
-  const float rinv = rcp_table[sb];           // f32(1 / f32(dec(sb) * gs)); entry 0 is 0
+  const float rinv = lds_f32(rcp_table + 4 * sb);   // f32(1 / f32(dec(sb) * gs)); entry 0 is 0
   const float2 rr = make_float2(rinv, rinv);
   float q0[8], q1[8];
 #pragma unroll
@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   const int m = m0 + qrow;
   const float c_x = __frcp_rn(__fmul_rn(6.0f, gs_x));
   const uint32_t KS4 = (uint32_t)(K >> 6);
+  const uint32_t rcp_u32 = smem_u32(s_rcp);
 
   float acc[Cfg::kAcc][4];
 #pragma unroll
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
     }
     const uint8_t* st = smem + s * Cfg::kStageBytes;
     const uint32_t st_u32 = smem_u32(st);
-    const float4* inv = reinterpret_cast<const float4*>(s_inv + s * 64 + 16 * qg);
+    const uint32_t inv_u32 = smem_u32(s_inv + s * 64 + 16 * qg);
 
     // ---- quantize two groups of row qrow ------------------------------------
     uint32_t w[4];
@@ -209,9 +210,12 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
       const int gg = qg + g;
-      const uint4 r0 = *reinterpret_cast<const uint4*>(st + sw128(qrow, 2 * gg));
-      const uint4 r1 = *reinterpret_cast<const uint4*>(st + sw128(qrow, 2 * gg + 1));
-      const uint32_t sb = quant_group(r0, r1, inv + 4 * g, c_x, s_rcp, w[2 * g], w[2 * g + 1]);
+      const uint4 r0 = lds_v4(st_u32 + sw128(qrow, 2 * gg));
+      const uint4 r1 = lds_v4(st_u32 + sw128(qrow, 2 * gg + 1));
+      float4 inv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) inv[j] = lds_v4f(inv_u32 + 64 * g + 16 * j);
+      const uint32_t sb = quant_group(r0, r1, inv, c_x, rcp_u32, w[2 * g], w[2 * g + 1]);
       sb2 |= sb << (8 * g);
     }
     const uint32_t other = __shfl_xor_sync(0xffffffffu, sb2, 1);
