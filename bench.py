@@ -39,6 +39,10 @@ FALLBACK_BF16_TFLOPS = 1590.0       # earlier measurement on this machine (burst)
 FALLBACK_HBM_GBS = 6650.0
 FP4_OVER_BF16 = 4.0                 # nominal dense ratio (9 / 2.25 PFLOP/s)
 N_COPIES = 4
+# DRAM bytes (read + write) of one k_linear launch from an ncu capture of this bench
+# (profiles/k_linear_qkv.md), valid only for the kernel sources it was taken on: the
+# sha256 prefix of csrc/linear.cuh + csrc/common.cuh.  Any other source -> traffic null.
+LINEAR_TRAFFIC = {"qkv": {"bytes": 27.004928e6 + 35.037184e6, "sources": "1d6510c42d96a3b8"}}
 
 
 def parse():
@@ -61,6 +65,20 @@ def peaks():
         return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+
+
+def linear_sources_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("linear.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "w4a4_rank_absorbed_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def linear_traffic(workload: str):
+    t = LINEAR_TRAFFIC.get(workload)
+    return t["bytes"] if t and t["sources"] == linear_sources_hash() else None
 
 
 def layer_flops(M, K, N, r):
@@ -208,7 +226,7 @@ def workload_config(wl):
             "M": wl.M, "K": wl.K, "N": wl.N, "r": wl.r_eff,
             "flops_per_step": layer_flops(wl.M, wl.K, wl.N, wl.r_eff),
             "l2": f"inputs larger than L2: the loop rotates over {N_COPIES} copies of the layer and its buffers",
-            "launch": "each kernel of a step replayed from a CUDA graph captured once per layer copy"}
+            "launch": "the timed steps replayed from one CUDA graph (2 kernel launches per step)"}
 
 
 # --------------------------------------------------------------- our arm -----
@@ -257,60 +275,94 @@ def run_ours(args):
         gemm(i)
     torch.cuda.synchronize()
 
-    # Each kernel launch of a step is captured once per layer copy in a CUDA graph; a timed step
-    # replays the copy's two graphs.  Replays take the host a few microseconds, so the launches
-    # queue ahead of the GPU and the step time is device time, not Python and ctypes overhead.
-    cap = torch.cuda.Stream(device=dev)
-    cap.wait_stream(torch.cuda.current_stream())
-    qa_graphs, ln_graphs = [], []
-    with torch.cuda.stream(cap):
-        for c in range(N_COPIES):
-            gq, gl = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gq, stream=cap):
-                quantize(c)
-            with torch.cuda.graph(gl, stream=cap):
-                gemm(c)
-            qa_graphs.append(gq)
-            ln_graphs.append(gl)
-    torch.cuda.current_stream().wait_stream(cap)
-    for i in range(max(args.warmup, N_COPIES)):
-        qa_graphs[i % N_COPIES].replay()
-        ln_graphs[i % N_COPIES].replay()
+    from w4a4_rank_absorbed_b200 import svdq as C
+
+    # The K timed steps are captured in one CUDA graph (step i: kernel 2 then kernel 3 on layer
+    # copy i % N_COPIES) and the timed region is one replay of it: device time, without the
+    # Python/ctypes launch overhead or the gaps between separately launched graphs.  The
+    # per-kernel averages come from two more graphs holding only kernel 2 or only kernel 3
+    # launches over the same copies, timed the same way right after.
+    def capture(fn, n):
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g, stream=cap):
+                for i in range(n):
+                    fn(i)
+        torch.cuda.current_stream().wait_stream(cap)
+        return g
+
+    def step(i):
+        quantize(i)
+        gemm(i)
+
+    n_kernel = 4 * N_COPIES
+    g_steps = capture(step, args.steps)
+    g_qa = capture(quantize, n_kernel)
+    g_ln = capture(gemm, n_kernel)
+    for g in (g_steps, g_qa, g_ln):        # warm replays, untimed
+        g.replay()
     torch.cuda.synchronize()
 
-    def step(i, ev):
-        ev[0].record()
-        qa_graphs[i % N_COPIES].replay()
-        ev[1].record()
-        ln_graphs[i % N_COPIES].replay()
-        ev[2].record()
+    def timed(g):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    t_start.record()
-    for i in range(args.steps):
-        step(i, evs[i])
-    t_end.record()
-    torch.cuda.synchronize()
+    ms = timed(g_steps) / args.steps
     if world > 1:
         dist.barrier()
+    t_qa = timed(g_qa) / n_kernel
+    t_ln = timed(g_ln) / n_kernel
     clk = clocks.stop()
-    from w4a4_rank_absorbed_b200 import svdq as C
     st, site = C.svdq_get_device_error()
     if st != 0:
         raise SystemExit(f"device error {st} at {site:#x}")
+    # The same layer without its low-rank branch (kernel 2 with r = 0, kernel 3 with r = 0) and
+    # with the branch unfused (down-projection X L1f and up-projection Y += LA L2 as separate
+    # cuBLAS calls that re-read X and re-read and re-write Y): the cost of the branch, fused and not.
 
-    ms = t_start.elapsed_time(t_end) / args.steps
-    t_qa = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    t_ln = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
-    ms, t_qa, t_ln = max_over_ranks([ms, t_qa, t_ln], device=dev)
-    del qa_graphs, ln_graphs
+    def plain(i):
+        L = layers[i % N_COPIES]
+        Xq, SFx, _ = L.act_buffers(M)
+        C.svdq_quantize_act(Xs[i % N_COPIES], M, K, L.inv_s, L.gs_x, None, 0, 1.0, Xq, SFx, None)
+        C.svdq_linear(Xq, SFx, L.gs_x, L.Wq, L.SFw, L.gs_w, None, None, 0, L.bias, Ys[i % N_COPIES], 0, M, N, K)
+
+    lr = []
+    for L in layers:
+        if r:
+            lr.append((L.L1fT.t().contiguous(), L.L2p[:, :r].t().contiguous(),
+                       torch.empty((M, r), dtype=torch.bfloat16, device=dev)))
+
+    def unfused(i):
+        plain(i)
+        if r:
+            L1f, L2b, LA = lr[i % N_COPIES]
+            torch.matmul(Xs[i % N_COPIES], L1f, out=LA)
+            Ys[i % N_COPIES].addmm_(LA, L2b)
+
+    for i in range(N_COPIES):              # eager first: creates the cuBLAS handle and workspace
+        unfused(i)
+    torch.cuda.synchronize()
+    g_plain = capture(plain, n_kernel)
+    g_unf = capture(unfused, n_kernel)
+    g_plain.replay()
+    g_unf.replay()
+    torch.cuda.synchronize()
+    t_plain = timed(g_plain) / n_kernel
+    t_unf = timed(g_unf) / n_kernel
+    ms, t_qa, t_ln, t_plain, t_unf = max_over_ranks([ms, t_qa, t_ln, t_plain, t_unf], device=dev)
+    del g_steps, g_qa, g_ln, g_plain, g_unf
 
     # end to end through the public API with host buffers (H2D of X, D2H of Y inside the timed region)
     Xh = X0.pin_memory()
@@ -346,13 +398,17 @@ def run_ours(args):
         "config": workload_config(wl),
         "pct_of_nvfp4_peak": 100.0 * (value / world) / fp4_peak,
         "roofline": {"bound": "tensor", "kernel": "svdq_linear (k_linear)", "achieved": lin_tf, "peak": fp4_peak,
-                     "unit": "TFLOP/s", "frac": lin_tf / fp4_peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": lin_tf / fp4_peak, "traffic": linear_traffic(args.workload),
                      "peak_source": f"{peak_kind} bf16 {bf16_peak:.1f} TFLOP/s x {FP4_OVER_BF16:.0f} (nominal "
                                     f"NVFP4:bf16 dense ratio)",
                      "flops_per_launch": lin_flops, "ms_per_launch": t_ln},
         "kernels": {"svdq_quantize_act": {"ms": t_qa, "GB_per_s": qa_gbs, "hbm_peak_GB_per_s": hbm_peak,
                                           "frac": qa_gbs / hbm_peak, "algorithmic_bytes": qa_bytes},
                     "svdq_linear": {"ms": t_ln, "TFLOP_per_s": lin_tf}},
+        "lowrank_branch": {"fused_ms_per_step": ms, "without_branch_ms_per_step": t_plain,
+                           "unfused_ms_per_step": t_unf, "fused_overhead": ms / t_plain - 1.0,
+                           "unfused_overhead": t_unf / t_plain - 1.0, "gate_fused_overhead": 0.15,
+                           "unfused": "kernel 2 and 3 at r = 0, then X L1f and Y += LA L2 as cuBLAS bf16 calls"},
         "clocks": clk,
         "e2e": {"value": job_throughput(fl, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 2), "ms_per_step": e2e_ms},
