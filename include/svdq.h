@@ -166,6 +166,11 @@ SVDQ_API svdq_status svdq_get_device_error(svdq_stream_t stream, int* site);
  * svdq_linear_debug -- svdq_linear with test hooks, for the fault-path tests.
  *   debug_flags bit 0: the load warp issues no loads, so the MMA warp's first
  *                      wait can never complete and must run out.
+ *               bit 1: use the single-CTA kernel (128 x 256 tiles) whatever M is.
+ *               bit 2: use the CTA-pair kernel (256 x 256 tiles) whatever M is.
+ *   (svdq_linear itself uses the single-CTA kernel; the CTA-pair kernel gives the same
+ *   results up to the fp32 accumulation order and is kept for comparison.  Setting both
+ *   bits 1 and 2 is SVDQ_ERR_INVALID_ARG.)
  *   timeout_ns: bound of every barrier wait (0 = the default of 2 s).
  * Otherwise identical to svdq_linear.
  */

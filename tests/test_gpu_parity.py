@@ -99,6 +99,30 @@ def test_linear_on_oracle_codes(M, N, K, r, use_bias, y_fp32):
     assert st == 0, site
 
 
+@pytest.mark.parametrize("kernel", ["single", "pair"])
+@pytest.mark.parametrize("M,N,K,r", [(256, 512, 512, 32), (100, 272, 576, 16), (520, 1296, 1536, 128),
+                                     (384, 144, 64, 0), (1, 16, 64, 48)])
+def test_linear_single_and_pair_kernels(M, N, K, r, kernel):
+    # svdq_linear picks the CTA-pair kernel for M > 128; force each kernel on every shape.
+    from w4a4_rank_absorbed_b200 import svdq as C
+    wl = small_case(M, K, N, r, seed=5 * M + N + K)
+    dec = oracle_layer(wl, r)
+    pw = OL.pack_weight(dec.R32)
+    qa = OL.quantize_act(wl.X, dec.inv_s, dec.gs_x, dec.L1f)
+    gs_x, gs_w = np.float32(dec.gs_x), pw.gs_w
+    lr_scale = np.float32(1.0 / (np.float64(gs_x) * np.float64(gs_w)))
+    Xq, SFx, Wq, SFw, LAs, L2p = _oracle_inputs_to_device(qa, pw, dec, lr_scale)
+    bias = bf16_dev(wl.bias)
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    flag = 2 if kernel == "single" else 4
+    C.svdq_linear_debug(Xq, SFx, float(gs_x), Wq, SFw, float(gs_w), LAs, L2p, r, bias, Y, 1, M, N, K, flag, 0)
+    torch.cuda.synchronize()
+    Y_or = OL.linear(qa, gs_x, pw, dec.L2b, wl.bias)
+    check_y(Y.cpu().numpy().astype(np.float64), Y_or, bf16=False, what=f"{kernel} Y {M}x{N}x{K} r={r}")
+    st, site = C.svdq_get_device_error()
+    assert st == 0, site
+
+
 @pytest.mark.parametrize("M,N,K,r", [(256, 512, 512, 32), (300, 528, 768, 16), (64, 256, 256, 0),
                                      (129, 400, 320, 64)])
 def test_layer_end_to_end(M, N, K, r):

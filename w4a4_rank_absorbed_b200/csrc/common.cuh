@@ -118,6 +118,35 @@ SVDQ_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, vol
   }
 }
 
+// mbar_wait for a barrier that also receives arrivals released at cluster scope by the other
+// CTA of a pair: the successful test acquires at cluster scope.
+SVDQ_DEV bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+SVDQ_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, volatile int* abort,
+                                unsigned site) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_cluster(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      *abort = 1;
+      report_timeout(site);
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA -----
 SVDQ_DEV void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");

@@ -63,7 +63,8 @@ static_assert(LN_SF_COL0 + LN_STAGES * LN_SF_COLS_PER_STAGE <= LN_TMEM_COLS, "TM
 static_assert(LN_STAGES * LN_STREAMS <= 32 && LN_STREAMS == 3, "one lane per slot and stream");
 static_assert(LN_REGS_LOW * 256 + LN_REGS_HIGH * 256 == LN_THREADS * 128, "register split = launch budget");
 
-enum : int { LN_DBG_NO_LOADS = 1 };
+// Test hooks (svdq_linear_debug): no loads (a forced time-out), force one kernel or the other.
+enum : int { LN_DBG_NO_LOADS = 1, LN_DBG_FORCE_SINGLE = 2, LN_DBG_FORCE_PAIR = 4 };
 
 #ifndef LN_RASTER_GM
 #define LN_RASTER_GM 12
@@ -92,6 +93,63 @@ struct LinearArgs {
   int debug;
   uint64_t timeout_ns;
 };
+
+// Epilogue store of one accumulator row: 128 columns from n0, y = f32(gs_x gs_w) acc + bias,
+// rounded to bf16 (or kept fp32 in test mode).  16 columns at a time: one 32-byte store of
+// bf16 (two of fp32); N % 16 == 0, so a group is either wholly inside the matrix or wholly
+// past its end.
+SVDQ_DEV void store_y_row(const LinearArgs& a, const uint32_t (&v)[4][32], int row, int n0, float gs) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int gp = 0; gp < 2; ++gp) {
+      const int n = n0 + 32 * i + 16 * gp;
+      if (n < a.N) {
+        float y[16];
+        if (a.bias) {
+          const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
+          const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 8));
+          const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            y[2 * e] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 2 * e]), bf16_lo(bw[e]));
+            y[2 * e + 1] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 2 * e + 1]), bf16_hi(bw[e]));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) y[e] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + e]), 0.0f);
+        }
+        if (a.y_fp32) {
+          float* dst = static_cast<float*>(a.Y) + (int64_t)row * a.N + n;
+          if (a.y_vec32) {
+            st_global_v8(dst, __float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                         __float_as_uint(y[3]), __float_as_uint(y[4]), __float_as_uint(y[5]),
+                         __float_as_uint(y[6]), __float_as_uint(y[7]));
+            st_global_v8(dst + 8, __float_as_uint(y[8]), __float_as_uint(y[9]), __float_as_uint(y[10]),
+                         __float_as_uint(y[11]), __float_as_uint(y[12]), __float_as_uint(y[13]),
+                         __float_as_uint(y[14]), __float_as_uint(y[15]));
+          } else {
+            float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d4[e] = make_float4(y[4 * e], y[4 * e + 1], y[4 * e + 2], y[4 * e + 3]);
+          }
+        } else {
+          uint32_t o[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+          uint16_t* dst = static_cast<uint16_t*>(a.Y) + (int64_t)row * a.N + n;
+          if (a.y_vec32) {
+            st_global_v8(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+        }
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     const __grid_constant__ CUtensorMap tm_xq,   // uint8 {K/2, M},  box {128, 128}, SW128
@@ -353,60 +411,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
       if (lane == 0) mbar_arrive(acc_empty);
 
       const int row = mb * LN_BM + 32 * q + lane;
-      if (row < M) {
-        // 16 columns at a time: one 32-byte store of bf16 (two of fp32); N % 16 == 0, so a
-        // group is either wholly inside the matrix or wholly past its end.
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-          for (int gp = 0; gp < 2; ++gp) {
-            const int n = nb * LN_BN + h * 128 + 32 * i + 16 * gp;
-            if (n < N) {
-              float y[16];
-              if (args.bias) {
-                const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
-                const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(args.bias + n + 8));
-                const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  y[2 * e] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 2 * e]), bf16_lo(bw[e]));
-                  y[2 * e + 1] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 2 * e + 1]), bf16_hi(bw[e]));
-                }
-              } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) y[e] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + e]), 0.0f);
-              }
-              if (args.y_fp32) {
-                float* dst = static_cast<float*>(args.Y) + (int64_t)row * N + n;
-                if (args.y_vec32) {
-                  st_global_v8(dst, __float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
-                               __float_as_uint(y[3]), __float_as_uint(y[4]), __float_as_uint(y[5]),
-                               __float_as_uint(y[6]), __float_as_uint(y[7]));
-                  st_global_v8(dst + 8, __float_as_uint(y[8]), __float_as_uint(y[9]), __float_as_uint(y[10]),
-                               __float_as_uint(y[11]), __float_as_uint(y[12]), __float_as_uint(y[13]),
-                               __float_as_uint(y[14]), __float_as_uint(y[15]));
-                } else {
-                  float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-                  for (int e = 0; e < 4; ++e) d4[e] = make_float4(y[4 * e], y[4 * e + 1], y[4 * e + 2], y[4 * e + 3]);
-                }
-              } else {
-                uint32_t o[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
-                uint16_t* dst = static_cast<uint16_t*>(args.Y) + (int64_t)row * N + n;
-                if (args.y_vec32) {
-                  st_global_v8(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
-                } else {
-                  uint4* d4 = reinterpret_cast<uint4*>(dst);
-                  d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                  d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
-                }
-              }
-            }
-          }
-        }
-      }
+      if (row < M) store_y_row(args, v, row, nb * LN_BN + h * 128, gs);
     }
   } else {
     regs_dec<LN_REGS_LOW>();                       // warp 3: no role

@@ -12,6 +12,7 @@
 #include "../../include/svdq.h"
 #include "common.cuh"
 #include "linear.cuh"
+#include "linear_pair.cuh"
 #include "pack_weight.cuh"
 #include "quantize_act.cuh"
 
@@ -27,6 +28,7 @@ struct DevInfo {
   bool ok = false;
   int sms = 0;
   bool linear_attr = false;
+  bool linear_pair_attr = false;
   bool qa_attr[9] = {};
 };
 DevInfo g_dev[kMaxDevices];
@@ -164,7 +166,16 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
     tm_las = tm_xq;
     tm_l2p = tm_wq;
   }
-  if (!d->linear_attr) {
+  // The single-CTA kernel by default.  The CTA-pair kernel (256 x 256 tiles, half of B per CTA)
+  // gives the same results but measured slower on B200 (0.118 against 0.075 ms on the QKV layer):
+  // the signals between the two CTAs sit on every stage's critical path.  Debug bit 2 selects it.
+  const bool pair = (debug & LN_DBG_FORCE_PAIR) != 0;
+  if (pair && !d->linear_pair_attr) {
+    if (cudaFuncSetAttribute(k_linear_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, LP_SMEM) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    d->linear_pair_attr = true;
+  }
+  if (!pair && !d->linear_attr) {
     if (cudaFuncSetAttribute(k_linear, cudaFuncAttributeMaxDynamicSharedMemorySize, LN_SMEM) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     d->linear_attr = true;
@@ -183,9 +194,15 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   a.gs = gs_x * gs_w;
   a.debug = debug;
   a.timeout_ns = timeout_ns ? timeout_ns : LN_DEFAULT_TIMEOUT_NS;
-  const int64_t tiles = ((M + LN_BM - 1) / LN_BM) * ((N + LN_BN - 1) / LN_BN);
-  const int grid = (int)(tiles < d->sms ? tiles : d->sms);
-  k_linear<<<grid, LN_THREADS, LN_SMEM, s>>>(tm_xq, tm_wq, tm_las, tm_l2p, a);
+  if (pair) {
+    const int64_t tiles = ((M + LP_BM - 1) / LP_BM) * ((N + LP_BN - 1) / LP_BN);
+    const int64_t pairs = tiles < d->sms / 2 ? tiles : d->sms / 2;
+    k_linear_pair<<<(int)(2 * pairs), LP_THREADS, LP_SMEM, s>>>(tm_xq, tm_wq, tm_las, tm_l2p, a);
+  } else {
+    const int64_t tiles = ((M + LN_BM - 1) / LN_BM) * ((N + LN_BN - 1) / LN_BN);
+    const int grid = (int)(tiles < d->sms ? tiles : d->sms);
+    k_linear<<<grid, LN_THREADS, LN_SMEM, s>>>(tm_xq, tm_wq, tm_las, tm_l2p, a);
+  }
   return launch_status();
 }
 
@@ -277,7 +294,9 @@ svdq_status svdq_linear_debug(const uint8_t* Xq, const uint8_t* SFx, float gs_x,
                               const uint8_t* SFw, float gs_w, const uint16_t* LAs, const uint16_t* L2p, int r,
                               const uint16_t* bias, void* Y, int y_fp32, int64_t M, int64_t N, int64_t K,
                               int debug_flags, uint64_t timeout_ns, svdq_stream_t stream) {
-  if (debug_flags & ~LN_DBG_NO_LOADS) return SVDQ_ERR_INVALID_ARG;
+  if ((debug_flags & ~(LN_DBG_NO_LOADS | LN_DBG_FORCE_SINGLE | LN_DBG_FORCE_PAIR)) ||
+      ((debug_flags & LN_DBG_FORCE_SINGLE) && (debug_flags & LN_DBG_FORCE_PAIR)))
+    return SVDQ_ERR_INVALID_ARG;
   return linear_impl(Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p, r, bias, Y, y_fp32, M, N, K, debug_flags, timeout_ns,
                      reinterpret_cast<cudaStream_t>(stream));
 }
