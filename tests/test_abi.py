@@ -67,8 +67,9 @@ def test_argument_errors_before_any_launch(lib):
         svdq.SVDQ_ERR_INVALID_ARG
     assert lib.svdq_pack_weight(16, 16, 128, 40, 32, 16, 16, 16, 16, None) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
     assert lib.svdq_pack_weight(4, 16, 128, 32, 32, 16, 16, 16, 16, None) == svdq.SVDQ_ERR_MISALIGNED
-    assert lib.svdq_linear_debug(16, 16, 1.0, 16, 16, 1.0, 16, 16, 32, None, 16, 0, 128, 256, 256, 4, 0, None) == \
-        svdq.SVDQ_ERR_INVALID_ARG
+    for flags in (8, 2 | 4):       # an unknown bit; both kernels forced at once
+        assert lib.svdq_linear_debug(16, 16, 1.0, 16, 16, 1.0, 16, 16, 32, None, 16, 0, 128, 256, 256, flags, 0,
+                                     None) == svdq.SVDQ_ERR_INVALID_ARG
 
 
 def test_valid_arguments_without_a_gpu_report_a_device_error(lib):
