@@ -57,8 +57,13 @@ def test_quantize_act_bitexact(M, K, r):
     g.check_errors()
 
 
-def _oracle_inputs_to_device(qa, pw, dec, lr_scale):
-    """The oracle's codes/scales and a hi/lo split of its float64 low-rank product, as device buffers."""
+def _oracle_inputs_to_device(qa, pw, dec, lr_scale, r_expected):
+    """The oracle's codes/scales and a hi/lo split of its float64 low-rank product, as device buffers.
+
+    The buffers are sized by the decomposition's rank, which the launch must use: a kernel
+    told a larger r would read past LAs and L2p.
+    """
+    assert dec.L1f.shape[1] == r_expected, f"decomposition rank {dec.L1f.shape[1]} != {r_expected}"
     Xq = torch.from_numpy(OC.pack_codes(qa.codes)).cuda()
     SFx = torch.from_numpy(sf_to_storage(qa.scales)).cuda()
     Wq = torch.from_numpy(OC.pack_codes(pw.codes)).cuda()
@@ -88,7 +93,7 @@ def test_linear_on_oracle_codes(M, N, K, r, use_bias, y_fp32):
     qa = OL.quantize_act(wl.X, dec.inv_s, dec.gs_x, dec.L1f)
     gs_x, gs_w = np.float32(dec.gs_x), pw.gs_w
     lr_scale = np.float32(1.0 / (np.float64(gs_x) * np.float64(gs_w)))
-    Xq, SFx, Wq, SFw, LAs, L2p = _oracle_inputs_to_device(qa, pw, dec, lr_scale)
+    Xq, SFx, Wq, SFw, LAs, L2p = _oracle_inputs_to_device(qa, pw, dec, lr_scale, r)
     bias = bf16_dev(wl.bias) if use_bias else None
     Y = torch.empty((M, N), dtype=torch.float32 if y_fp32 else torch.bfloat16, device="cuda")
     C.svdq_linear(Xq, SFx, float(gs_x), Wq, SFw, float(gs_w), LAs, L2p, r, bias, Y, int(y_fp32), M, N, K)
@@ -101,7 +106,7 @@ def test_linear_on_oracle_codes(M, N, K, r, use_bias, y_fp32):
 
 @pytest.mark.parametrize("kernel", ["single", "pair"])
 @pytest.mark.parametrize("M,N,K,r", [(256, 512, 512, 32), (100, 272, 576, 16), (520, 1296, 1536, 128),
-                                     (384, 144, 64, 0), (1, 16, 64, 48)])
+                                     (384, 144, 64, 0), (1, 64, 128, 48)])
 def test_linear_single_and_pair_kernels(M, N, K, r, kernel):
     # svdq_linear picks the CTA-pair kernel for M > 128; force each kernel on every shape.
     from w4a4_rank_absorbed_b200 import svdq as C
@@ -111,7 +116,7 @@ def test_linear_single_and_pair_kernels(M, N, K, r, kernel):
     qa = OL.quantize_act(wl.X, dec.inv_s, dec.gs_x, dec.L1f)
     gs_x, gs_w = np.float32(dec.gs_x), pw.gs_w
     lr_scale = np.float32(1.0 / (np.float64(gs_x) * np.float64(gs_w)))
-    Xq, SFx, Wq, SFw, LAs, L2p = _oracle_inputs_to_device(qa, pw, dec, lr_scale)
+    Xq, SFx, Wq, SFw, LAs, L2p = _oracle_inputs_to_device(qa, pw, dec, lr_scale, r)
     bias = bf16_dev(wl.bias)
     Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
     flag = 2 if kernel == "single" else 4
