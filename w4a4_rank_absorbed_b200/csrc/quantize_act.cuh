@@ -9,16 +9,22 @@
 // diag(s)^-1 L1, so X L1f = X_hat L1) on the tensor cores (bf16 in, fp32
 // accumulate), pre-scaled by lr_scale and split into bf16 hi/lo halves.
 //
-// CTA = 32 rows x all of K; 14 consumer warps in 7 pairs + 1 TMA producer warp.
-// The K axis is cut into 64-column chunks; chunk c goes through ring stage
-// c % S and is consumed by warp pair c % 7, so seven chunks are processed at
-// once and up to S loads are in flight (S = 14, or 7 for r > 88; S is a multiple of 7).  A stage holds the X box (32 x 64
-// bf16, 128-byte swizzle), the L1f^T box (r x 64 bf16, same swizzle) and the
-// chunk's 64 smoothing factors.  Warp h of a pair owns rows 16h..16h+15
-// of the chunk: two lanes per row quantize two groups of 16 each, and the
-// warp runs the 16 x r down-projection of its rows for the chunk's 64 columns
-// (mma.sync m16n8k16), keeping a partial sum in registers.  After the last
-// chunk the seven partial sums of every row are added in shared memory and
+// CTA = 32 rows x all of K; 14 warps in 7 pairs.  The K axis is cut into
+// 64-column chunks; chunk c goes through ring stage c % S and is consumed by
+// warp pair c % 7, so seven chunks are processed at once.  S is a multiple of
+// 7 (up to 49): as many stages as fit in 200 KB, 21 for r = 32, 7 for r = 128,
+// so each pair keeps S/7 chunks in flight.  A pair loads its own chunks: once
+// both of its warps are done with a stage, warp 0 of the pair issues the copies
+// of the chunk S further on into that stage (three lanes in one converged
+// instruction, rotating with the round so no thread has two copies in flight:
+// a thread's copies are serviced one after another).  No producer warp, and no
+// lanes waiting on different barriers in divergent branches.  A stage holds
+// the X box (32 x 64 bf16, 128-byte swizzle), the L1f^T box (r x 64 bf16, same
+// swizzle) and the chunk's 64 smoothing factors.  Warp h of a pair owns rows
+// 16h..16h+15 of the chunk: two lanes per row quantize two groups of 16 each,
+// and the warp runs the 16 x r down-projection of its rows for the chunk's 64
+// columns (mma.sync m16n8k16), keeping a partial sum in registers.  After the
+// last chunk the seven partial sums of every row are added in shared memory and
 // written as LAs.
 #pragma once
 #include "common.cuh"
@@ -29,7 +35,7 @@ constexpr int QA_ROWS = 32;
 constexpr int QA_CHUNK = 64;          // bf16 columns per chunk (128 bytes)
 constexpr int QA_PAIRS = 7;
 constexpr int QA_CONSUMER_WARPS = 2 * QA_PAIRS;
-constexpr int QA_THREADS = (QA_CONSUMER_WARPS + 1) * 32;
+constexpr int QA_THREADS = QA_CONSUMER_WARPS * 32;
 constexpr int QA_RING_BYTES = 200 * 1024;
 
 template <int R>
@@ -37,10 +43,10 @@ struct QaCfg {
   static constexpr int kXBytes = QA_ROWS * 128;
   static constexpr int kLBytes = R * 128;
   static constexpr int kStageBytes = kXBytes + kLBytes;
-  // The ring size is a multiple of the pair count, so a ring slot is always consumed by the
-  // same warp pair and its rounds are waited for in order (a parity wait cannot tell round r
-  // from round r - 2).
-  static constexpr int kStages = (2 * QA_PAIRS * kStageBytes <= QA_RING_BYTES) ? 2 * QA_PAIRS : QA_PAIRS;
+  // The ring size is a multiple of the pair count, so a ring slot is always loaded and consumed
+  // by the same warp pair, one round after another.
+  static constexpr int kPerPair = QA_RING_BYTES / (QA_PAIRS * (kStageBytes + 256));
+  static constexpr int kStages = QA_PAIRS * (kPerPair < 1 ? 1 : kPerPair > 7 ? 7 : kPerPair);
   static constexpr int kNT = R / 8;                                  // n8 tiles of the r columns
   static constexpr int kAcc = R > 0 ? kNT : 1;                      // (m16, n8) tiles per warp
   static constexpr int kRedBytes = QA_PAIRS * QA_ROWS * R * 4;
@@ -131,18 +137,20 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   float* s_inv = reinterpret_cast<float*>(smem + Cfg::kInvOff);
   float* s_rcp = reinterpret_cast<float*>(smem + Cfg::kRcpOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
-  uint64_t* empty = full + S;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S);
+  uint64_t* consumed = full + S;           // both warps of the owning pair are done with the stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(consumed + S);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * QA_ROWS;
   const int nchunks = K / QA_CHUNK;
+  const int pairi = warp >> 1;             // warp pair: consumes chunks pairi, pairi + 7, ...
+  const int half = warp & 1;               // rows 16*half .. 16*half + 15 of the chunk
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 2);
+      mbar_init(&consumed[s], 2);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -152,36 +160,35 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
     const uint32_t sb = threadIdx.x;
     s_rcp[sb] = sb == 0 ? 0.0f : __frcp_rn(__fmul_rn(dec_ue4m3(sb), gs_x));
   }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    if (R > 0) tma_prefetch_desc(&tm_l1);
+  }
   __syncthreads();
 
-  if (warp == QA_CONSUMER_WARPS) {
-    // ---------------------------------------------------------- producer --
-    // Lane 2g + k serves ring slot g (chunks c with c % S == g) and stream k (0: X box,
-    // 1: L1f^T box and the chunk's 64 smoothing factors).  A thread's TMA copies are
-    // serviced one after another, so each lane keeps at most two copies in flight.
-    const int g = lane >> 1, k = lane & 1;
-    if (g < S) {
-      if (lane == 0) tma_prefetch_desc(&tm_x);
-      if (lane == 1 && R > 0) tma_prefetch_desc(&tm_l1);
-      for (int c = g; c < nchunks; c += S) {
-        const uint32_t parity = (uint32_t)((c / S) & 1);
-        if (!mbar_wait(&empty[g], parity ^ 1u, timeout_ns, abort_flag, 0x201)) break;
-        uint8_t* st = smem + g * Cfg::kStageBytes;
-        if (k == 0) {
-          mbar_arrive_expect_tx(&full[g], Cfg::kStageBytes + 256);
-          tma_load_2d(st, &tm_x, &full[g], c * QA_CHUNK, m0);
-        } else {
-          if (R > 0) tma_load_2d(st + Cfg::kXBytes, &tm_l1, &full[g], c * QA_CHUNK, 0);
-          bulk_load(s_inv + g * 64, inv_s + (int64_t)c * QA_CHUNK, 256, &full[g]);
-        }
-      }
+  // Copies of chunk c into its stage, by lanes 3j .. 3j + 2 of warp 0 of the owning pair (j
+  // rotates with the round): X box and L1f^T box in one converged instruction, then the chunk's
+  // 64 smoothing factors.
+  auto issue = [&](int c) {
+    const int g = c % S;
+    const int j = (c / S) % 10;
+    if (lane >= 3 * j && lane < 3 * j + 3) {
+      const int k = lane - 3 * j;
+      uint8_t* st = smem + g * Cfg::kStageBytes;
+      if (k == 0) mbar_arrive_expect_tx(&full[g], Cfg::kStageBytes + 256);
+      __syncwarp(7u << (3 * j));
+      if (k == 0 || (k == 1 && R > 0))
+        tma_load_2d(k == 0 ? st : st + Cfg::kXBytes, k == 0 ? &tm_x : &tm_l1, &full[g], c * QA_CHUNK,
+                    k == 0 ? m0 : 0);
+      else if (k == 2)
+        bulk_load(s_inv + g * 64, inv_s + (int64_t)c * QA_CHUNK, 256, &full[g]);
     }
-    return;
-  }
+    __syncwarp();
+  };
+  int hi = pairi;                          // the pair's chunks below hi have been issued
+  for (; hi < nchunks && hi < S; hi += QA_PAIRS)
+    if (half == 0) issue(hi);
 
-  // -------------------------------------------------------------- consumers --
-  const int pairi = warp >> 1;             // warp pair: consumes chunks pairi, pairi + 7, ...
-  const int half = warp & 1;               // rows 16*half .. 16*half + 15 of the chunk
   const int qrow = 16 * half + (lane >> 1);
   const int qg = 2 * (lane & 1);           // first of the two groups this lane quantizes
   const int m = m0 + qrow;
@@ -194,7 +201,8 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
   for (int i = 0; i < Cfg::kAcc; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
 
   bool ok = true;
-  for (int c = pairi; c < nchunks; c += QA_PAIRS) {
+  int c = pairi;
+  for (; c < nchunks; c += QA_PAIRS) {
     const int s = c % S;
     if (!mbar_wait(&full[s], (uint32_t)((c / S) & 1), timeout_ns, abort_flag, 0x202)) {
       ok = false;
@@ -242,8 +250,30 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
         }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    // Once both warps of the pair are done with stage s, warp 0 refills it with the chunk S
+    // further on.
+    if (c + S < nchunks) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&consumed[s]);
+      if (half == 0) {
+        int done = 1;
+        if (lane == 0) done = mbar_wait(&consumed[s], (uint32_t)((c / S) & 1), timeout_ns, abort_flag, 0x201) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, done, 0)) {
+          ok = false;
+          c += QA_PAIRS;                   // chunk c was consumed; the loads still owed start after it
+          break;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(c + S);
+      }
+      hi = c + S + QA_PAIRS;
+    }
+  }
+  if (!ok && half == 0) {
+    // Let the loads this pair issued but did not consume land before the CTA exits.
+    int never = 0;
+    for (int c2 = c; c2 < hi; c2 += QA_PAIRS)
+      mbar_wait(&full[c2 % S], (uint32_t)((c2 / S) & 1), timeout_ns, &never, 0x203);
   }
 
   // ---- LAs = [hi | lo] of lr_scale * sum over pairs of the partial X L1f ----
