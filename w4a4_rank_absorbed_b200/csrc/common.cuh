@@ -1,5 +1,5 @@
 // Device helpers shared by the SVDQuant kernels: inline PTX for mbarriers,
-// TMA, tcgen05 (TMEM, MMA, copies) and the FP4/FP8 conversions.
+// TMA, tcgen05 (TMEM allocation, MMA, loads and stores) and the FP4/FP8 conversions.
 // Written for sm_100a from the public PTX ISA.
 #pragma once
 
@@ -53,8 +53,6 @@ SVDQ_DEV uint64_t globaltimer_ns() {
   return t;
 }
 
-SVDQ_DEV uint32_t lane_id() { return threadIdx.x & 31u; }
-
 // ------------------------------------------------------------- mbarrier -----
 SVDQ_DEV void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -85,18 +83,6 @@ SVDQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test: has the phase with parity `parity` completed?
-SVDQ_DEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 
 // Wait for the phase with parity `parity` to complete.  Gives up after
 // `timeout_ns` of wall time, or as soon as `*abort` is set by another role of
@@ -197,12 +183,6 @@ SVDQ_DEV void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar, in
       ::"r"(smem_u32(dst)), "l"(m), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
-SVDQ_DEV void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t bar, int32_t x, int32_t y, int32_t z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-      ::"r"(smem_u32(dst)), "l"(m), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
 
 SVDQ_DEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -240,9 +220,6 @@ SVDQ_DEV void tc_mma_bf16_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint3
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
-}
-SVDQ_DEV void tc_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // -------------------------------------------------------------- tcgen05 -----
@@ -286,11 +263,6 @@ SVDQ_DEV void tc_mma_bf16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t i
       : "memory");
 }
 
-// Copy a 32-row x 16-byte shared-memory block into TMEM lanes 0-31 (4 columns)
-// and replicate it into the other three lane quarters.
-SVDQ_DEV void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
 
 // Each thread of the warp reads 32 consecutive 32-bit columns of its TMEM lane.
 SVDQ_DEV void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
@@ -328,12 +300,6 @@ SVDQ_DEV void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::
 template <int N>
 SVDQ_DEV void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 
-SVDQ_DEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t x, int32_t y, int32_t z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-      ::"r"(smem_u32(dst)), "l"(m), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
-}
 
 SVDQ_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -358,13 +324,6 @@ SVDQ_DEV uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
-// Shared-memory descriptor of a 32-row x 16-byte scale block (no swizzle, rows contiguous).
-SVDQ_DEV uint64_t sdesc_sf_block(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)(128u >> 4) << 32;   // 8-row groups 128 bytes apart
-  d |= (uint64_t)1u << 46;
-  return d;
-}
 
 // Instruction descriptor, kind::mxf4nvf4: A, B = E2M1 (K-major), scales UE4M3, M x N, dense K = 64.
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
