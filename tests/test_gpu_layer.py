@@ -1,0 +1,63 @@
+"""The packed-layer API (SVDQLinear) on the GPU: device forward, host-buffer forward and the
+streamed host-buffer path agree with each other bit for bit and with the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import OL, check_y, require_gpu
+from w4a4_rank_absorbed_b200.synth import small_case
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _layer(M, K, N, r, seed):
+    from w4a4_rank_absorbed_b200.calib import calibrate
+    from w4a4_rank_absorbed_b200.layer import SVDQLinear
+    wl = small_case(M, K, N, r, seed=seed)
+    data = calibrate(wl.X, wl.W, r, 0.5, bias=wl.bias)
+    return wl, data, SVDQLinear(data, device=torch.device("cuda", 0))
+
+
+def test_forward_matches_oracle_and_host_paths():
+    M, K, N, r = 300, 512, 528, 32
+    wl, data, L = _layer(M, K, N, r, seed=41)
+    X = torch.from_numpy(wl.X.astype(np.float32)).to(torch.bfloat16)
+    Y_dev = L.forward(X.cuda()).cpu()
+    # oracle on the same layer constants (the layer's own decomposition, its packed weight)
+    inv_s = data.inv_s.double().numpy()
+    L1f = data.L1fT.t().float().double().numpy()
+    L2b = data.L2b.float().double().numpy()
+    Y_or, _, _ = OL.svdq_reference(X.float().double().numpy(), inv_s, data.gs_x, L1f, L2b,
+                                   data.R.numpy(), data.bias.float().double().numpy())
+    check_y(Y_dev.float().numpy().astype(np.float64), Y_or, bf16=True, what="layer forward")
+
+    Xh = X.pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xd, Yd = torch.empty((M, K), dtype=torch.bfloat16, device="cuda"), torch.empty((M, N), dtype=torch.bfloat16,
+                                                                                    device="cuda")
+    L.forward_host(Xh, Yh, Xd, Yd)
+    torch.cuda.synchronize()
+    assert torch.equal(Yh, Y_dev)
+
+
+def test_streamed_host_batches_match_forward():
+    M, K, N, r = 256, 256, 272, 16
+    wl, data, L = _layer(M, K, N, r, seed=43)
+    g = torch.Generator().manual_seed(7)
+    Xs = [(torch.randn((M, K), generator=g) * (1.0 + 0.5 * i)).to(torch.bfloat16) for i in range(5)]
+    want = [L.forward(X.cuda()).cpu() for X in Xs]
+    Xh = [X.pin_memory() for X in Xs]
+    Yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in Xs]
+    X_devs = [torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    Y_devs = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    L.forward_host_stream(Xh, Yh, X_devs, Y_devs)
+    torch.cuda.synchronize()
+    for i in range(len(Xs)):
+        assert torch.equal(Yh[i], want[i]), f"batch {i}"
+    from w4a4_rank_absorbed_b200 import svdq as C
+    assert C.svdq_get_device_error()[0] == 0

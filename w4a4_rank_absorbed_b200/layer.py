@@ -89,3 +89,42 @@ class SVDQLinear:
         X_dev.copy_(X_host, non_blocking=True)
         self.forward(X_dev, out=Y_dev)
         Y_host.copy_(Y_dev, non_blocking=True)
+
+    def forward_host_stream(self, X_hosts, Y_hosts, X_devs, Y_devs) -> None:
+        """A sequence of host batches through the layer, copies overlapped with compute.
+
+        Batch i: its X (pinned host) is copied in on one stream, the two kernels run on a second,
+        its Y is copied out (to pinned host) on a third, so batch i+1's copy in and batch i-1's
+        copy out overlap batch i's kernels.  X_devs / Y_devs are two (or more) device buffers used
+        in turn; a buffer is refilled only after the batch that used it has left it.  Asynchronous
+        with respect to the host; events order the streams.
+        """
+        nb = len(X_devs)
+        cur = torch.cuda.current_stream(self.device)
+        s_in, s_cmp, s_out = (torch.cuda.Stream(device=self.device) for _ in range(3))
+        for st in (s_in, s_cmp, s_out):
+            st.wait_stream(cur)
+        done_cmp = [None] * nb
+        done_out = [None] * nb
+        for i, (Xh, Yh) in enumerate(zip(X_hosts, Y_hosts)):
+            b = i % nb
+            with torch.cuda.stream(s_in):
+                if done_cmp[b] is not None:
+                    s_in.wait_event(done_cmp[b])          # the kernels that read X_devs[b] are done
+                X_devs[b].copy_(Xh, non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in)
+                if done_out[b] is not None:
+                    s_cmp.wait_event(done_out[b])         # Y_devs[b] has been copied out
+                self.forward(X_devs[b], out=Y_devs[b], stream=s_cmp)
+                done_cmp[b] = torch.cuda.Event()
+                done_cmp[b].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done_cmp[b])
+                Yh.copy_(Y_devs[b], non_blocking=True)
+                done_out[b] = torch.cuda.Event()
+                done_out[b].record(s_out)
+        for st in (s_in, s_cmp, s_out):
+            cur.wait_stream(st)
