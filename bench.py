@@ -42,7 +42,7 @@ N_COPIES = 4
 # DRAM bytes (read + write) of one k_linear launch from an ncu capture of this bench
 # (profiles/k_linear_qkv.md), valid only for the kernel sources it was taken on: the
 # sha256 prefix of csrc/linear.cuh + csrc/common.cuh.  Any other source -> traffic null.
-LINEAR_TRAFFIC = {"qkv": {"bytes": 26.584320e6 + 38.115072e6, "sources": "ed582377a869d9af"}}
+LINEAR_TRAFFIC = {"qkv": {"bytes": 26.841600e6 + 35.598336e6, "sources": "126cf5ca30aee97e"}}
 
 
 def parse():
