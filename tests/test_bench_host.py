@@ -1,0 +1,43 @@
+"""Host-side logic of the bench and the build (no GPU): FLOP count, traffic bookkeeping, the
+register check that guards the setmaxnreg split, and the JSON config."""
+import bench
+from w4a4_rank_absorbed_b200 import build
+from w4a4_rank_absorbed_b200.synth import make_workload
+
+
+def test_layer_flops_counts_gemm_and_both_projections():
+    M, K, N, r = 4608, 3072, 9216, 32
+    assert bench.layer_flops(M, K, N, r) == 2.0 * M * N * K + 2.0 * M * r * K + 2.0 * M * r * N
+    assert bench.layer_flops(M, K, N, 0) == 2.0 * M * N * K
+
+
+def test_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
+    h = bench.linear_sources_hash()
+    assert len(h) == 16
+    monkeypatch.setattr(bench, "LINEAR_TRAFFIC", {"qkv": {"bytes": 123.0, "sources": h}})
+    assert bench.linear_traffic("qkv") == 123.0
+    assert bench.linear_traffic("large") is None
+    monkeypatch.setattr(bench, "LINEAR_TRAFFIC", {"qkv": {"bytes": 123.0, "sources": "0" * 16}})
+    assert bench.linear_traffic("qkv") is None
+
+
+def test_entry_register_parser():
+    log = "\n".join([
+        "ptxas info    : Compiling entry function '_ZN4svdq13k_linear_pairE14CUtensorMap_st' for 'sm_100a'",
+        "ptxas info    : Function properties for _ZN4svdq13k_linear_pairE14CUtensorMap_st",
+        "    8 bytes stack frame, 4 bytes spill stores, 8 bytes spill loads",
+        "ptxas info    : Used 128 registers, used 0 barriers",
+        "ptxas info    : Compiling entry function '_ZN4svdq8k_linearE14CUtensorMap_st' for 'sm_100a'",
+        "ptxas info    : Used 120 registers, used 1 barriers",
+    ])
+    assert build.entry_registers(log, "13k_linear_pairE") == 128
+    assert build.entry_registers(log, "8k_linearE") == 120
+    assert build.entry_registers(log, "k_missing") is None
+
+
+def test_workload_config_names_the_workload_and_sizes():
+    wl = make_workload("tiny")
+    cfg = bench.workload_config(wl)
+    assert cfg["workload"].startswith("tiny")
+    assert (cfg["M"], cfg["K"], cfg["N"], cfg["r"]) == (wl.M, wl.K, wl.N, wl.r_eff)
+    assert "L2" in cfg["l2"] and "graph" in cfg["launch"]
