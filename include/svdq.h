@@ -40,8 +40,12 @@
  *     a launch failure returns SVDQ_ERR_CUDA.  Kernel-side faults that do not
  *     stop the kernel (a bounded wait that ran out) are reported by
  *     svdq_get_device_error().
- *   - Pointers must be 16-byte aligned.  Shapes: K % 64 == 0, N % 16 == 0,
- *     r % 16 == 0 with 0 <= r <= 128, 1 <= M, K, N < 2^31.  Any M.
+ *   - Pointers must be 16-byte aligned (svdq_linear stores Y 32 bytes at a time
+ *     when Y is 32-byte aligned, 16 bytes otherwise).  Shapes: K % 64 == 0,
+ *     N % 16 == 0, r % 16 == 0 with 0 <= r <= 128, 1 <= M, K, N < 2^31.  Any M.
+ *   - Buffer sizes cannot be checked from pointers: every buffer must hold the
+ *     shape the call states (a larger r than LAs / L2p were sized for makes the
+ *     kernels read past them).
  *   - One device per call: the current device of the calling thread.
  *     Requires compute capability 10.0 (B200, sm_100a).
  */
