@@ -287,7 +287,9 @@ def run_ours(args):
         cap = torch.cuda.Stream(device=dev)
         cap.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(cap):
-            with torch.cuda.graph(g, stream=cap):
+            # thread_local: under torchrun the process group's watchdog thread queries CUDA events
+            # while we capture; the default (global) mode would invalidate the capture.
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
                 for i in range(n):
                     fn(i)
         torch.cuda.current_stream().wait_stream(cap)
