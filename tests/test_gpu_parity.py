@@ -84,7 +84,9 @@ def _oracle_inputs_to_device(qa, pw, dec, lr_scale, r_expected):
 @pytest.mark.parametrize("M,N,K,r,use_bias", [(256, 512, 512, 32, True), (200, 400, 320, 16, True),
                                               (128, 256, 64, 0, False), (384, 768, 1024, 32, True),
                                               (70, 144, 256, 64, False), (129, 272, 576, 48, True),
-                                              (1, 16, 64, 16, True), (520, 1296, 1536, 128, True)])
+                                              (1, 16, 64, 16, True), (520, 1296, 1536, 128, True),
+                                              (128, 128, 128, 0, True), (256, 256, 128, 16, False),
+                                              (128, 256, 64, 16, True)])
 def test_linear_on_oracle_codes(M, N, K, r, use_bias, y_fp32):
     from w4a4_rank_absorbed_b200 import svdq as C
     wl = small_case(M, K, N, r, seed=M + 3 * N + K)
@@ -162,7 +164,8 @@ def test_tiny_config_and_method_effect():
 
 def test_edge_values():
     # all-zero rows and groups, negative zeros, values at E2M1 ties, and a calibration scale that makes
-    # some runtime groups saturate their UE4M3 scale (gs_x calibrated on smaller activations).
+    # some runtime groups saturate their UE4M3 scale (gs_x calibrated on smaller activations), others
+    # fall to subnormal scales or to a zero scale.
     M, K, N, r = 96, 256, 64, 16
     wl = small_case(M, K, N, r, seed=123)
     X = wl.X.copy()
@@ -172,13 +175,17 @@ def test_edge_values():
     X[11, :16] = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, -0.25, -0.75, -1.25, -1.75, -2.5, -3.5, -5.0,
                            -6.0])
     X[13, :] *= 1e4
-    dec = OD.decompose(X, wl.W, r, 0.5, X_cal=wl.X)     # calibrated without the scaled row
+    X[15, :] *= 1e-4            # block scales in the UE4M3 subnormal range
+    X[17, :] *= 1e-7            # block scales that round to 0: all codes 0
+    dec = OD.decompose(X, wl.W, r, 0.5, X_cal=wl.X)     # calibrated without the scaled rows
     X = np.asarray(torch.from_numpy(X).to(torch.bfloat16).double().numpy())
     g = GpuLayer(dec, wl.bias)
     Xq, SFx, LAs = g.quantize(bf16_dev(X))
     qa = OL.quantize_act(X, dec.inv_s, dec.gs_x, dec.L1f)
     ref = oracle_storage(qa=qa)
     assert (qa.scales[13] == 0x7E).any(), "expected saturating scales in row 13"
+    assert ((qa.scales[15] > 0) & (qa.scales[15] < 8)).any(), "expected subnormal scales in row 15"
+    assert (qa.scales[17] == 0).all(), "expected zero scales in row 17"
     _assert_bytes(Xq, ref["Xq"], "Xq")
     _assert_bytes(SFx, ref["SFx"], "SFx")
     check_las(LAs, X, dec.L1f, g.lr_scale)
