@@ -13,9 +13,10 @@
 //
 // Per CTA (16 warps, same roles as k_linear):
 //   warp 0      tensor producer: A box (own 128 rows) and B box (own 128 rows of N), 128-byte
-//               swizzle.  The copies of both CTAs count on the first CTA's "full" barrier,
-//               whose one arrival (with the expected bytes of both CTAs) comes from the first
-//               CTA's producer.
+//               swizzle, counted on the CTA's own "full" barrier.  (Pair-form copies counted on
+//               the first CTA's barrier landed 3.7 us after issue against 1.1-1.4 us for local
+//               ones.)
+//   warp 3      in the second CTA: forwards each stage's "full" to the first CTA's "peer_full".
 //   warp 1      TMEM owner (cta_group::2 allocation); in the first CTA the MMA issuer: 4 MMAs
 //               of 256 x 256 x 64 per K tile, then the rank tiles; each commit is multicast to
 //               the "empty" barrier of both CTAs.
@@ -63,14 +64,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LP_THREADS, 1) k_lin
   uint8_t* sB = smem + LP_OFF_B;
   uint8_t* sSFA = smem + LP_OFF_SFA;
   uint8_t* sSFB = smem + LP_OFF_SFB;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + LP_OFF_BAR);   // both CTAs' A/B landed (first CTA)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + LP_OFF_BAR);   // this CTA's A/B landed
   uint64_t* sf_full = full + LP_STAGES;                               // this CTA's scale blocks landed
   uint64_t* sf_ready = sf_full + LP_STAGES;                           // both CTAs' scales in TMEM (first CTA)
   uint64_t* empty = sf_ready + LP_STAGES;                             // stage consumed by the MMAs
   uint64_t* acc_full = empty + LP_STAGES;
   uint64_t* acc_empty = acc_full + 1;                                 // first CTA: both epilogues done
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* peer_full = drain + 1;                                    // first CTA: the other CTA's A/B landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_full + LP_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -96,6 +98,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LP_THREADS, 1) k_lin
       mbar_init(&sf_full[s], 1);
       mbar_init(&sf_ready[s], 8);                  // 4 scale writers in each CTA
       mbar_init(&empty[s], 1);
+      mbar_init(&peer_full[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * LN_EPI_WARPS);
@@ -118,8 +121,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LP_THREADS, 1) k_lin
       // --------------------------------------------------------- producers --
       // In-order, warp-uniform waits on this CTA's "empty" (multicast by the first CTA's
       // commits); lane S g + k issues stream k of slot g, the stage's lanes in one converged
-      // instruction.  Warp 0: k = 0 A, 1 B (pair-form copies counted on the first CTA's
-      // "full").  Warp 2: k = 0 SFA, 1 SFB block 0, 2 SFB block 1 (this CTA's "sf_full").
+      // instruction.  Warp 0: k = 0 A, 1 B (this CTA's "full").  Warp 2: k = 0 SFA, 1 SFB
+      // block 0, 2 SFB block 1 (this CTA's "sf_full").
       const bool tensor_warp = warp == 0;
       const int per = tensor_warp ? 2 : 3;
       const int g = lane / per, k = lane % per;
@@ -151,14 +154,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LP_THREADS, 1) k_lin
           const unsigned smask = (tensor_warp ? 3u : 7u) << (per * stage);
           if (tensor_warp) {
             if (mine) {
-              if (k == 0 && rank == 0)
-                mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (LP_A_BYTES + LP_B_BYTES)));
-              const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+              if (k == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(LP_A_BYTES + LP_B_BYTES));
               const CUtensorMap* map = k == 0 ? (lr ? &tm_las : &tm_xq) : (lr ? &tm_l2p : &tm_wq);
               uint8_t* dst = k == 0 ? sA + stage * LP_A_BYTES : sB + stage * LP_B_BYTES;
               const int x = lr ? (kt - nkt) * 64 : kt * 128;
               __syncwarp(smask);
-              tma_load_2d_pair(dst, map, fb, x, k == 0 ? arow : brow);
+              tma_load_2d(dst, map, &full[stage], x, k == 0 ? arow : brow);
               issued = true;
               last_parity = phase;
             }
@@ -185,12 +186,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LP_THREADS, 1) k_lin
         }
       }
       if (*abort_flag && issued) {
-        // Let this lane's last copy land before the CTA exits.  A pair-form copy is counted on
-        // the first CTA's barrier; the first CTA waits there, the other CTA relies on the final
-        // cluster barrier, which the first CTA reaches only after its own wait.
+        // Let this lane's last copy land before the CTA exits.
         int never = 0;
-        if (!tensor_warp) mbar_wait(&sf_full[g], last_parity, tmo, &never, 0x402);
-        else if (rank == 0) mbar_wait(&full[g], last_parity, tmo, &never, 0x402);
+        mbar_wait(tensor_warp ? &full[g] : &sf_full[g], last_parity, tmo, &never, 0x402);
       }
     }
   } else if (warp == 1) {
@@ -208,6 +206,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LP_THREADS, 1) k_lin
         tc_fence_after();
         for (int kt = 0; kt < nst; ++kt) {
           if (!mbar_wait(&full[stage], phase, tmo, abort_flag, 0x412) ||
+              !mbar_wait_cluster(&peer_full[stage], phase, tmo, abort_flag, 0x415) ||
               !mbar_wait_cluster(&sf_ready[stage], phase, tmo, abort_flag, 0x414)) {
             ok = false;
             break;
@@ -310,7 +309,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LP_THREADS, 1) k_lin
       if (row < M) store_y_row(args, v, row, nb * LP_BN + h * 128, gs);
     }
   } else {
-    regs_dec<LN_REGS_LOW>();                       // warp 3: no role
+    regs_dec<LN_REGS_LOW>();
+    // warp 3 of the second CTA: forwards "this CTA's A/B of the stage landed" to the first CTA
+    if (rank == 1 && lane == 0) {
+      const uint32_t peer0 = mapa_shared(smem_u32(peer_full), 0);
+      int gi = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs)
+        for (int kt = 0; kt < nst; ++kt, ++gi) {
+          const int st2 = gi % LP_STAGES;
+          if (!mbar_wait(&full[st2], (uint32_t)((gi / LP_STAGES) & 1), tmo, abort_flag, 0x441)) { ok = false; break; }
+          mbar_arrive_cluster(peer0 + 8u * (uint32_t)st2);
+        }
+    }
   }
 
   // Both CTAs leave together: TMEM is allocated for the pair and arrivals cross between them.
