@@ -1,5 +1,4 @@
 """The C ABI library loads, exports every declared symbol and validates arguments (CPU only)."""
-import ctypes
 import os
 import re
 

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import (GpuLayer, OC, OD, OL, bf16_dev, bf16_host, check_las, check_y, mismatch_report,
+from helpers import (GpuLayer, OC, OD, OL, bf16_dev, check_las, check_y, mismatch_report,
                      oracle_storage, require_gpu, u8_host)
 from oracle.layout import sf_offsets
 from w4a4_rank_absorbed_b200.synth import make_workload

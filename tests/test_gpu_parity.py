@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import (GpuLayer, OC, OD, OL, bf16_bits, bf16_dev, bf16_host, check_las, check_y, f32_dev,
+from helpers import (GpuLayer, OC, OD, OL, bf16_dev, bf16_host, check_las, check_y,
                      mismatch_report, oracle_layer, oracle_storage, require_gpu, u8_host)
 from oracle.layout import sf_to_storage
 from w4a4_rank_absorbed_b200.synth import make_workload, small_case
