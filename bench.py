@@ -449,7 +449,7 @@ def run_ours(args):
         "gpu_launches": 2 * args.steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = args.cpu_sample_rows or 1024
+        rows = min(args.cpu_sample_rows or M, M)       # default: every row of the step (a few s of CPU)
         out["cpu_baseline"] = cpu_baseline(wl, rows)
     if rank == 0:
         print(json.dumps(out), flush=True)
