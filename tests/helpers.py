@@ -58,13 +58,15 @@ def half_ulp_bf16(y: np.ndarray) -> np.ndarray:
 
 
 def check_y(Y_gpu: np.ndarray, Y_or: np.ndarray, bf16: bool, what: str = ""):
-    """Output gate.  fp32 output: rel-Frobenius <= 2e-3 and max-abs <= 1e-2 rms(Y_or), literally.
-    bf16 output (one final rounding that no bf16 result can avoid): rel-Frobenius <= 2e-3 against the
-    oracle rounded to bf16, and max-abs <= 1e-2 rms(Y_or) + half a bf16 ulp of Y_or."""
+    """Output gate against the unrounded float64 oracle.
+
+    rel-Frobenius ||Y - Y_or||_F / ||Y_or||_F <= 2e-3 in both output modes (the bf16 rounding of the
+    output alone costs about 1.7e-3 of it, which is why the low-rank branch is carried as a hi/lo pair).
+    max-abs: fp32 output <= 1e-2 rms(Y_or); bf16 output <= 1e-2 rms(Y_or) + half a bf16 ulp of Y_or,
+    since rounding a value near 4 sigma to bf16 alone moves it by up to 1.6e-2 rms."""
     d = np.abs(Y_gpu - Y_or)
     rms = float(np.sqrt(np.mean(Y_or ** 2)))
-    ref = OD.bf16_round(Y_or) if bf16 else Y_or
-    rel = float(np.linalg.norm(Y_gpu - ref) / np.linalg.norm(Y_or))
+    rel = float(np.linalg.norm(Y_gpu - Y_or) / np.linalg.norm(Y_or))
     bound = MAX_ABS_RMS * rms + (half_ulp_bf16(Y_or) if bf16 else 0.0)
     worst = float(np.max(d - bound))
     assert rel <= REL_FRO, f"{what} rel-Frobenius {rel:.3e} > {REL_FRO}"
@@ -92,15 +94,16 @@ class GpuLayer:
         self.Wq = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
         self.SFw = torch.full((C.svdq_sf_bytes(N, K),), 0xAB, dtype=torch.uint8, device="cuda")
         self.gs_w_dev = torch.empty(1, dtype=torch.float32, device="cuda")
-        self.L2p = torch.empty((N, 2 * r), dtype=torch.bfloat16, device="cuda") if r else None
-        C.svdq_pack_weight(self.R, self.L2b, K, N, r, self.Wq, self.SFw, self.gs_w_dev, self.L2p)
-        torch.cuda.synchronize()
-        self.gs_w = np.float32(self.gs_w_dev.item())
+        self.L2p = torch.empty((N, r), dtype=torch.bfloat16, device="cuda") if r else None
+        self.gs_w = np.float32(C.svdq_pack_weight(self.R, self.L2b, K, N, r, self.Wq, self.SFw, self.gs_w_dev,
+                                                  self.L2p))
+        assert self.gs_w == np.float32(self.gs_w_dev.item())
         self.gs_x = np.float32(dec.gs_x)
         self.lr_scale = np.float32(1.0 / (np.float64(self.gs_x) * np.float64(self.gs_w)))
         self.inv_s = f32_dev(dec.inv_s)
         self.L1fT = bf16_dev(np.ascontiguousarray(dec.L1f.T)) if r else None
         self.bias = bf16_dev(bias) if bias is not None else None
+        self.ws = {}
 
     def quantize(self, X_dev):
         C = self.C
@@ -108,8 +111,10 @@ class GpuLayer:
         Xq = torch.empty((M, self.K // 2), dtype=torch.uint8, device="cuda")
         SFx = torch.full((C.svdq_sf_bytes(M, self.K),), 0xAB, dtype=torch.uint8, device="cuda")
         LAs = torch.empty((M, 2 * self.r), dtype=torch.bfloat16, device="cuda") if self.r else None
+        if M not in self.ws:
+            self.ws[M] = C.new_workspace(M, self.K, self.r)
         C.svdq_quantize_act(X_dev, M, self.K, self.inv_s, float(self.gs_x), self.L1fT, self.r,
-                            float(self.lr_scale), Xq, SFx, LAs)
+                            float(self.lr_scale), Xq, SFx, LAs, self.ws[M])
         return Xq, SFx, LAs
 
     def linear(self, Xq, SFx, LAs, y_fp32=False, bias=True):
@@ -128,10 +133,23 @@ def la_bound(X, L1f, lr_scale):
     return LA_REL * float(lr_scale) * (np.abs(X) @ np.abs(L1f))
 
 
+def las_split(las: np.ndarray, r: int):
+    """(hi, lo) of an LAs buffer (M x 2r, hi and lo interleaved by 16 columns)."""
+    g = las.reshape(las.shape[0], r // 16, 2, 16)
+    return g[:, :, 0, :].reshape(-1, r), g[:, :, 1, :].reshape(-1, r)
+
+
+def las_join(hi: np.ndarray, lo: np.ndarray) -> np.ndarray:
+    """The LAs layout from its hi and lo halves (M x r each): interleaved by 16 columns."""
+    M, r = hi.shape
+    return np.stack([hi.reshape(M, r // 16, 16), lo.reshape(M, r // 16, 16)], axis=2).reshape(M, 2 * r)
+
+
 def check_las(LAs_gpu: torch.Tensor, X, L1f, lr_scale, rows=None):
     r = L1f.shape[1]
     las = bf16_host(LAs_gpu)
-    v = las[:, :r] + las[:, r:]
+    hi, lo = las_split(las, r)
+    v = hi + lo
     Xs = X if rows is None else X[rows]
     if rows is not None:
         v = v[rows]
@@ -140,7 +158,6 @@ def check_las(LAs_gpu: torch.Tensor, X, L1f, lr_scale, rows=None):
     bound = la_bound(Xs, L1f, lr_scale) + 1e-30
     assert np.all(err <= bound), f"LAs error {float(np.max(err / bound)):.3f} of bound"
     # hi is the bf16 rounding of v: |lo| <= half an ulp of hi
-    hi, lo = las[:, :r], las[:, r:]
     assert np.all(np.abs(lo) <= half_ulp_bf16(hi) * 1.0000001 + 1e-38)
 
 

@@ -1,8 +1,9 @@
 """Parity at the full workload sizes, in the launch configuration the benchmark times.
 
-The whole weight is packed and compared byte for byte; activations, the
-down-projection and the output are compared on a sample of rows (the
-first, the last and random ones), which the oracle computes one by one.
+Every byte of the packed weight and of the quantized activations is compared
+with the oracle, the low-rank product on every row, and the layer output on
+every element, once with bf16 output and once with fp32 output (the oracle
+does a FLUX-sized layer in a few seconds).
 """
 import numpy as np
 import pytest
@@ -10,7 +11,6 @@ import torch
 
 from helpers import (GpuLayer, OC, OD, OL, bf16_dev, check_las, check_y, mismatch_report,
                      oracle_storage, require_gpu, u8_host)
-from oracle.layout import sf_offsets
 from w4a4_rank_absorbed_b200.synth import make_workload
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -21,40 +21,28 @@ def _gpu():
     require_gpu()
 
 
-def _rows(M, seed=0, n=96):
-    rng = np.random.default_rng(seed)
-    rows = set(range(min(8, M))) | set(range(max(0, M - 8), M)) | set(rng.choice(M, size=min(n, M), replace=False))
-    return np.array(sorted(rows))
-
-
-def _check_layer(wl, dec, X, what, y_rows_check=True):
+def _check_layer(wl, dec, X, what):
     g = GpuLayer(dec, wl.bias)
     M, K = X.shape
     Xq, SFx, LAs = g.quantize(bf16_dev(X))
-    Y = g.linear(Xq, SFx, LAs)
+    Y16 = g.linear(Xq, SFx, LAs)
+    Y32 = g.linear(Xq, SFx, LAs, y_fp32=True)
     torch.cuda.synchronize()
     g.check_errors()
-    # weight: every byte
     pw = OL.pack_weight(dec.R32)
+    qa = OL.quantize_act(X, dec.inv_s, dec.gs_x, dec.L1f)
     assert g.gs_w == pw.gs_w
-    ref = oracle_storage(pw=pw)
-    for name, buf in (("Wq", g.Wq), ("SFw", g.SFw)):
+    ref = oracle_storage(qa=qa, pw=pw)
+    for name, buf in (("Wq", g.Wq), ("SFw", g.SFw), ("Xq", Xq), ("SFx", SFx)):
         a, b = u8_host(buf), ref[name]
         assert np.array_equal(a, b), f"{what} {name}: " + mismatch_report(a, b)
-    # activations on sampled rows
-    rows = _rows(M, seed=M + K)
-    qa = OL.quantize_act(X[rows], dec.inv_s, dec.gs_x, dec.L1f)
-    xq = Xq.cpu().numpy()[rows]
-    assert np.array_equal(xq, OC.pack_codes(qa.codes)), f"{what} Xq"
-    sfx = u8_host(SFx)[sf_offsets(M, K // 16)[rows]]
-    assert np.array_equal(sfx, qa.scales), f"{what} SFx"
     if dec.L1f.shape[1]:
-        las = LAs.cpu()[rows]
-        check_las(las, X[rows], dec.L1f, g.lr_scale)
+        check_las(LAs.cpu(), X, dec.L1f, g.lr_scale)
     Y_or = OL.linear(qa, dec.gs_x, pw, dec.L2b, wl.bias)
-    Yg = Y.float().cpu().numpy()[rows].astype(np.float64)
-    rel, mx = check_y(Yg, Y_or, bf16=True, what=what)
-    return g, Y, rel, mx
+    rel16, mx16 = check_y(Y16.float().cpu().numpy().astype(np.float64), Y_or, bf16=True, what=what + " bf16")
+    rel32, mx32 = check_y(Y32.cpu().numpy().astype(np.float64), Y_or, bf16=False, what=what + " fp32")
+    print(f"{what}: bf16 rel-Fro {rel16:.3e} max/rms {mx16:.3e}; fp32 rel-Fro {rel32:.3e} max/rms {mx32:.3e}")
+    return g, Y16
 
 
 def test_qkv_projection():
@@ -72,7 +60,7 @@ def test_large_batch():
 def test_mlp_pair_fc1_gelu_fc2():
     wl1 = make_workload("fc1")
     dec1 = OD.decompose(wl1.X, wl1.W, wl1.r, wl1.alpha)
-    _, Y1, _, _ = _check_layer(wl1, dec1, wl1.X, "fc1")
+    _, Y1 = _check_layer(wl1, dec1, wl1.X, "fc1")
     # GELU (tanh form) on the harness side; fc2 is calibrated on and compared on this same bf16 tensor
     X2 = torch.nn.functional.gelu(Y1.float(), approximate="tanh").to(torch.bfloat16)
     X2 = X2.double().cpu().numpy()

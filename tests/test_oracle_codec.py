@@ -81,12 +81,41 @@ def test_ue4m3_saturates():
     assert (ue4m3_encode(v) == 0x7E).all()
 
 
-def test_global_scale():
+def _nearest_f32(q):
+    """The float32 nearest to the positive rational q (ties to even), found by exact rational search."""
+    from fractions import Fraction
+    q = Fraction(q)
+    e = q.numerator.bit_length() - q.denominator.bit_length()
+    while Fraction(2) ** e > q:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= q:
+        e += 1
+    ulp = Fraction(2) ** (max(e, -126) - 23)           # normal (or subnormal) spacing at q
+    k, rem = divmod(q, ulp)
+    if rem * 2 > ulp or (rem * 2 == ulp and k % 2 == 1):
+        k += 1
+    return F32(float(k * ulp))
+
+
+def test_global_scale_closed_forms():
+    # amax = 2688 * 2^k gives exactly 2^k; 2688 = 21 * 2^7, so amax = 21 gives 2^-7
+    for k in range(-30, 31):
+        assert global_scale(F32(2688.0 * 2.0 ** k)) == F32(2.0 ** k)
+    assert global_scale(F32(21.0)) == F32(2.0 ** -7)
+    assert global_scale(F32(8064.0)) == F32(3.0)
     assert global_scale(0.0) == F32(1.0)
-    assert global_scale(2688.0) == F32(1.0)
-    assert global_scale(F32(3.0)) == F32(F32(3.0) / F32(2688.0))
     with pytest.raises(ValueError):
         global_scale(np.inf)
+
+
+def test_global_scale_is_the_correctly_rounded_quotient():
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    amaxes = np.concatenate([[F32(3.0), F32(7.0), F32(1e-30), F32(6.0e4)],
+                             np.exp(rng.uniform(-20, 20, 2000)).astype(F32)])
+    for a in amaxes:
+        want = _nearest_f32(Fraction(float(a)) / 2688)
+        assert global_scale(a) == want, (a, global_scale(a), want)
 
 
 def _grid_tensor(rng, rows, K, gs):

@@ -95,3 +95,47 @@ def test_sf_layout_is_a_bijection():
     o = sf_offsets(128, 4)
     assert o[0, 0] == 0 and o[1, 0] == 16 and o[32, 0] == 4 and o[33, 3] == 16 + 4 + 3 and o[127, 3] == 511
     assert sf_offsets(128, 8)[0, 4] == 512 and sf_offsets(256, 4)[128, 0] == 512
+
+
+def test_activation_global_scale_hand_built():
+    # f32(X * inv_s) is exact here (powers of two), and the largest magnitude sits at a known
+    # negative entry of a column whose smoothing factor enlarges it: amax = 168 * 4 = 672 -> 672/2688 = 1/4.
+    X = np.zeros((6, 32))
+    X[:, :] = 1.5
+    X[3, 5] = -168.0
+    X[0, 7] = 500.0                      # larger raw value, but its channel is shrunk by 1/8
+    inv_s = np.ones(32, dtype=np.float32)
+    inv_s[5] = 4.0
+    inv_s[7] = 0.125
+    assert D.activation_global_scale(X, inv_s) == np.float32(0.25)
+    # without the smoothing the raw maximum 500 would decide: 500/2688 is a different scale
+    assert D.activation_global_scale(X, np.ones(32, dtype=np.float32)) != np.float32(0.25)
+    # all-zero activations: scale 1
+    assert D.activation_global_scale(np.zeros((4, 16)), np.ones(16, dtype=np.float32)) == np.float32(1.0)
+
+
+def test_activation_global_scale_rounds_the_product_to_float32_first():
+    # x = 2688 (a bf16 value), inv_s = 1 + 2^-20: the exact product 2688 + 10.5 * 2^-12 is a tie at
+    # float32's spacing 2^-12 and rounds to 2688 + 10 * 2^-12, so gs_x must come from the product
+    # rounded to float32 first, then divided by 2688.
+    s = np.float32(1.0 + 2.0 ** -20)
+    X = np.full((2, 16), 2688.0)
+    from w4a4_rank_absorbed_b200.synth import round_to_bf16
+    assert round_to_bf16(X[0, 0]) == X[0, 0]
+    inv_s = np.full(16, s, dtype=np.float32)
+    got = D.activation_global_scale(X, inv_s)
+    # f32(2709 (1 + 2^-20)) = 2709 + 2709 * 2^-20 rounded to float32's spacing 2^-12 at 2709
+    from fractions import Fraction
+    exact = Fraction(2688) * (1 + Fraction(1, 2 ** 20))
+    spacing = Fraction(1, 2 ** 12)
+    k, rem = divmod(exact, spacing)
+    if rem * 2 > spacing or (rem * 2 == spacing and k % 2 == 1):
+        k += 1
+    prod32 = k * spacing
+    assert float(prod32) != float(exact)          # the rounding step matters in this case
+    q = prod32 / 2688
+    sp = Fraction(1, 2 ** 23)                      # q is in [1, 2)
+    k2, rem2 = divmod(q, sp)
+    if rem2 * 2 > sp or (rem2 * 2 == sp and k2 % 2 == 1):
+        k2 += 1
+    assert got == np.float32(float(k2 * sp))
