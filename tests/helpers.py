@@ -14,6 +14,7 @@ from oracle.layout import sf_to_storage
 REL_FRO = 2e-3          # ||Y - Y_or||_F / ||Y_or||_F
 MAX_ABS_RMS = 1e-2      # max |Y - Y_or| <= 1e-2 rms(Y_or)   (+ half a bf16 ulp of Y_or for bf16 output)
 LA_REL = 2e-5           # |LAs_hi + LAs_lo - lr_scale X L1f| <= 2e-5 lr_scale (|X| |L1f|)
+REL_ROUNDED_MARGIN = 1e-4   # bf16 output: rel-Frobenius may exceed the rounded oracle's own by this much
 
 
 def require_gpu():
@@ -67,9 +68,16 @@ def check_y(Y_gpu: np.ndarray, Y_or: np.ndarray, bf16: bool, what: str = ""):
     d = np.abs(Y_gpu - Y_or)
     rms = float(np.sqrt(np.mean(Y_or ** 2)))
     rel = float(np.linalg.norm(Y_gpu - Y_or) / np.linalg.norm(Y_or))
+    rel_bound = REL_FRO
+    if bf16:
+        # The best any bf16 output can do is the correctly rounded oracle; on outputs of a few dozen
+        # elements its own rel-Frobenius can exceed 2e-3 (2.05e-3 on a 1 x 16 output), so the bound
+        # is never below that figure plus a small margin for the float32 arithmetic.
+        rho = float(np.linalg.norm(OD.bf16_round(Y_or) - Y_or) / np.linalg.norm(Y_or))
+        rel_bound = max(REL_FRO, rho + REL_ROUNDED_MARGIN)
     bound = MAX_ABS_RMS * rms + (half_ulp_bf16(Y_or) if bf16 else 0.0)
     worst = float(np.max(d - bound))
-    assert rel <= REL_FRO, f"{what} rel-Frobenius {rel:.3e} > {REL_FRO}"
+    assert rel <= rel_bound, f"{what} rel-Frobenius {rel:.3e} > {rel_bound:.3e}"
     assert worst <= 0, f"{what} max-abs error exceeds bound by {worst:.3e} (rms {rms:.3e})"
     return rel, float(d.max() / rms)
 
