@@ -2,21 +2,30 @@
 """Benchmark of the fused SVDQuant W4A4 linear layer on B200 (one process per GPU).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qkv] [--impl ours|reference]
+                    [--extra fc1,fc2,large] [--strong]
 
 A step is one forward pass of the layer over one batch: svdq_quantize_act
 (smoothing, NVFP4 encode, fused down-projection) then svdq_linear (NVFP4
 tcgen05 GEMM with the fused up-projection and bias).  The residual weight is
-packed once beforehand (it is static per layer).  To keep the L2 cache cold
-between steps, the timed loop rotates over 4 independent copies of the layer
-and of its input/output buffers (together several times the 126 MB L2).
+packed once beforehand (it is static per layer).  Between steps the L2 cache
+is kept cold by rotating over 4 independent copies of the layer and of its
+input/output buffers (together several times the 126 MB L2).
 
-Metric: TFLOP/s of the layer, counting 2MNK + 2Mr(K+N) per step, and the
-fraction of the NVFP4 dense tensor peak.  Under torchrun each rank runs the
-same layer on its own batch (weak scaling, no collective on the data path);
-the step time is the maximum over ranks.
+Headline: TFLOP/s of the layer on the FLUX QKV projection, counting
+2MNK + 2Mr(K+N) per step, over exactly K steps replayed from one CUDA graph.
+Every other time (the kernels alone, the layer without its low-rank branch,
+the in-house unfused pipeline, L2-warm and L2-flushed steps, the other FLUX
+shapes) comes from one protocol: a CUDA graph of S launches, replayed R times,
+each replay timed with CUDA events; the line reports the median and the 10th
+and 90th percentiles of the per-launch time.
 
---impl reference times the CPU oracle (test infrastructure) on a bounded
-sample of the same workload; rank 0 only.
+Under torchrun each rank runs its own replica of the layer (no collective on
+the data path): by default each rank processes its own batch of M rows (weak
+scaling); with --strong one batch of M rows is split into row blocks, one per
+rank (strong scaling).  Step times are the maximum over ranks.
+
+--impl reference times the CPU oracle (test infrastructure) on the same
+workload; rank 0 only.
 """
 from __future__ import annotations
 
@@ -39,22 +48,29 @@ FALLBACK_BF16_TFLOPS = 1590.0       # earlier measurement on this machine (burst)
 FALLBACK_HBM_GBS = 6650.0
 FP4_OVER_BF16 = 4.0                 # nominal dense ratio (9 / 2.25 PFLOP/s)
 N_COPIES = 4
-# DRAM bytes (read + write) of one k_linear launch from an ncu capture of this bench
-# (profiles/k_linear_qkv.md), valid only for the kernel sources it was taken on: the
-# sha256 prefix of csrc/linear.cuh + csrc/common.cuh.  Any other source -> traffic null.
-LINEAR_TRAFFIC = {"qkv": {"bytes": 26.841600e6 + 35.598336e6, "sources": "126cf5ca30aee97e"}}
+GRAPH_LAUNCHES = 20                 # S: launches (or steps) per timed graph
+GRAPH_REPLAYS = 50                  # R: timed replays per graph
+FLUSH_BYTES = 256 << 20             # written between steps of the L2-flushed leg (L2 is 126 MB)
+# DRAM bytes (read + write) of one k_linear launch on the QKV layer from an ncu capture, valid only
+# for the kernel sources it was taken on (sha256 prefix of csrc/linear.cuh + csrc/common.cuh);
+# any other source -> traffic null.
+LINEAR_TRAFFIC = {}
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default="qkv")
+    p.add_argument("--extra", default="fc1,fc2,large",
+                   help="other FLUX-sized workloads measured with the same protocol ('' for none)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--cpu-sample-rows", type=int, default=0, help="oracle rows per step (0 = auto)")
+    p.add_argument("--strong", action="store_true", help="split one batch of M rows across the ranks")
+    p.add_argument("--cpu-sample-rows", type=int, default=0, help="oracle rows (0 = every row of the batch)")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    return p.parse_args()
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args(argv)
 
 
 def peaks():
@@ -86,6 +102,37 @@ def layer_flops(M, K, N, r):
     return 2.0 * M * N * K + 2.0 * M * r * (K + N)
 
 
+def linear_flops(M, K, N, r):
+    """Work of kernel 3 alone: the 4-bit GEMM and the up-projection."""
+    return 2.0 * M * N * K + 2.0 * M * N * r
+
+
+def quantize_bytes(M, K, r):
+    """Algorithmic bytes of kernel 2: X read once, codes, scales, the low-rank product (bf16)."""
+    return 2.0 * M * K + M * K / 2 + M * K / 16 + 2.0 * M * r
+
+
+def unfused_extra_bytes(M, K, N, r):
+    """What the unfused pipeline moves on top of the fused one: X read again by the separate
+    down-projection, and Y read and written again by the separate up-projection (bf16)."""
+    return 2.0 * M * K + 4.0 * M * N
+
+
+def row_block(M: int, rank: int, world: int):
+    """Rows [lo, hi) of a batch of M rows that rank `rank` of `world` takes (contiguous, sizes differ by
+    at most one)."""
+    lo = rank * M // world
+    hi = (rank + 1) * M // world
+    return lo, hi
+
+
+def stats(samples):
+    """Median and 10th / 90th percentiles of a list of times (ms)."""
+    a = np.sort(np.asarray(samples, dtype=np.float64))
+    return {"median": float(np.median(a)), "p10": float(np.percentile(a, 10)), "p90": float(np.percentile(a, 90)),
+            "n": int(a.size)}
+
+
 def max_over_ranks(values, device=None):
     """Element-wise maximum of a list of floats over all ranks (identity without a process group)."""
     import torch
@@ -98,8 +145,21 @@ def max_over_ranks(values, device=None):
 
 
 def job_throughput(flops_per_rank_step, world, ms_per_step_max):
-    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's step time (weak scaling)."""
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's step time."""
     return flops_per_rank_step * world / (ms_per_step_max * 1e-3) / 1e12
+
+
+def cpu_cores():
+    """Host cores (nproc) and the BLAS thread count the oracle's float64 products run on."""
+    nproc = os.cpu_count() or 1
+    blas = None
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=None)
+    except Exception:
+        pass
+    return nproc, blas
 
 
 # --------------------------------------------------------------- clocks ------
@@ -135,6 +195,10 @@ class ClockSampler:
         rows = [l.strip().split(",") for l in self.file.read().splitlines() if l.strip()]
         self.file.close()
         os.unlink(self.file.name)
+        return self.summarize(rows)
+
+    @staticmethod
+    def summarize(rows):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
@@ -151,39 +215,29 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ oracle arm -----
-def oracle_forward_sample(wl, rows: int):
-    """Time the oracle's forward (quantize_act + linear) on the first `rows` rows; weight packed beforehand."""
+def oracle_forward(dec, pw, X, bias):
+    from oracle import linear as OL
+    qa = OL.quantize_act(X, dec.inv_s, dec.gs_x, dec.L1f)
+    return OL.linear(qa, dec.gs_x, pw, dec.L2b, bias)
+
+
+def oracle_setup(wl):
     from oracle import decompose as OD
     from oracle import linear as OL
     dec = OD.decompose(wl.X, wl.W, wl.r, wl.alpha, wl.lora_A, wl.lora_B)
-    pw = OL.pack_weight(dec.R32)
-    X = wl.X[:rows]
-    t0 = time.perf_counter()
-    qa = OL.quantize_act(X, dec.inv_s, dec.gs_x, dec.L1f)
-    OL.linear(qa, dec.gs_x, pw, dec.L2b, wl.bias)
-    dt = time.perf_counter() - t0
-    return dt, dec, pw
-
-
-def cpu_cores():
-    try:
-        import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        n = max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=None)
-        if n:
-            return int(n)
-    except Exception:
-        pass
-    return os.cpu_count() or 1
+    return dec, OL.pack_weight(dec.R32)
 
 
 def cpu_baseline(wl, rows: int):
-    dt, _, _ = oracle_forward_sample(wl, rows)
+    dec, pw = oracle_setup(wl)
+    t0 = time.perf_counter()
+    oracle_forward(dec, pw, wl.X[:rows], wl.bias)
+    dt = time.perf_counter() - t0
     fl = layer_flops(rows, wl.K, wl.N, wl.r_eff)
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"oracle forward (quantize_act + linear, float64 from dequantized values) of the first "
-                      f"{rows} of {wl.M} rows of the {wl.name} layer, weight packed beforehand; "
-                      f"{dt:.2f} s"}
+    nproc, blas = cpu_cores()
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": nproc, "blas_threads": blas, "kind": "oracle",
+            "sample": f"oracle forward (quantize_act + linear, float64 from dequantized values) of {rows} of "
+                      f"{wl.M} rows of the {wl.name} layer, weight packed beforehand; {dt:.2f} s"}
 
 
 def run_reference(args):
@@ -192,44 +246,230 @@ def run_reference(args):
         return
     from w4a4_rank_absorbed_b200.synth import make_workload
     wl = make_workload(args.workload)
-    rows = args.cpu_sample_rows or 256
-    from oracle import decompose as OD
-    from oracle import linear as OL
-    dec = OD.decompose(wl.X, wl.W, wl.r, wl.alpha, wl.lora_A, wl.lora_B)
-    pw = OL.pack_weight(dec.R32)
+    dec, pw = oracle_setup(wl)
+    # Each step is the oracle's forward over `rows` rows of the batch, every row by default (the same
+    # sample as the cpu_baseline of our arm); fewer when K + W steps of the whole batch would take more
+    # than about 150 s.
+    rows = min(args.cpu_sample_rows or wl.M, wl.M)
+    t0 = time.perf_counter()
+    oracle_forward(dec, pw, wl.X[:rows], wl.bias)
+    t_one = time.perf_counter() - t0
+    budget = 150.0
+    if (args.steps + args.warmup) * t_one > budget:
+        rows = max(128, int(rows * budget / ((args.steps + args.warmup) * t_one)))
     times = []
     for i in range(args.warmup + args.steps):
         lo = (i * rows) % max(1, wl.M - rows + 1)
-        X = wl.X[lo:lo + rows]
         t0 = time.perf_counter()
-        qa = OL.quantize_act(X, dec.inv_s, dec.gs_x, dec.L1f)
-        OL.linear(qa, dec.gs_x, pw, dec.L2b, wl.bias)
+        oracle_forward(dec, pw, wl.X[lo:lo + rows], wl.bias)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
-    dt = float(np.mean(times))
+    dt = float(np.median(times))
     fl = layer_flops(rows, wl.K, wl.N, wl.r_eff)
     val = fl / dt / 1e12
+    nproc, blas = cpu_cores()
     sample = f"oracle forward of {rows} of {wl.M} rows of the {wl.name} layer per step (weight packed beforehand)"
     out = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": workload_config(wl),
-           "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-                            "sample": sample},
+           "config": workload_config(wl, args),
+           "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": nproc, "blas_threads": blas,
+                            "kind": "oracle", "sample": sample},
            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
-def workload_config(wl):
+def workload_config(wl, args=None):
+    strong = bool(args and getattr(args, "strong", False))
     return {"workload": f"{wl.name}: SVDQuant linear M={wl.M} K={wl.K} N={wl.N} r={wl.r_eff} alpha={wl.alpha}, "
                         f"NVFP4 group 16, bf16 in/out",
             "M": wl.M, "K": wl.K, "N": wl.N, "r": wl.r_eff,
             "flops_per_step": layer_flops(wl.M, wl.K, wl.N, wl.r_eff),
             "l2": f"inputs larger than L2: the loop rotates over {N_COPIES} copies of the layer and its buffers",
-            "launch": "the timed steps replayed from one CUDA graph (2 kernel launches per step)"}
+            "launch": "the timed steps replayed from one CUDA graph (2 kernel launches per step)",
+            "ranks": "one batch of M rows split into row blocks across ranks" if strong else
+                     "each rank runs its own batch of M rows (replicas, no collective)"}
 
 
 # --------------------------------------------------------------- our arm -----
+class Timer:
+    """Capture a function of the launch index into a CUDA graph of S launches and time its replays."""
+
+    def __init__(self, torch, dev):
+        self.torch = torch
+        self.dev = dev
+
+    def capture(self, fn, n):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device=self.dev)
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            # thread_local: under torchrun the process group's watchdog thread queries CUDA events
+            # while we capture; the default (global) mode would invalidate the capture.
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+                for i in range(n):
+                    fn(i)
+        torch.cuda.current_stream().wait_stream(cap)
+        return g
+
+    def replay_ms(self, g):
+        torch = self.torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    def per_launch(self, fn, n=GRAPH_LAUNCHES, reps=GRAPH_REPLAYS):
+        g = self.capture(fn, n)
+        g.replay()
+        self.torch.cuda.synchronize()
+        samples = [self.replay_ms(g) / n for _ in range(reps)]
+        del g
+        return samples
+
+
+def build_layer_set(name, dev, rows=None, fc1_layer=None):
+    """Layer copies and buffers of one workload (calibrated on its own batch)."""
+    import torch
+
+    from w4a4_rank_absorbed_b200 import svdq as C
+    from w4a4_rank_absorbed_b200.calib import calibrate
+    from w4a4_rank_absorbed_b200.layer import SVDQLinear
+    from w4a4_rank_absorbed_b200.synth import make_workload
+
+    wl = make_workload(name)
+    if name == "fc2":
+        # fc2's input is GELU-tanh of fc1's output (the MLP pair), computed here on the GPU
+        Y1 = fc1_layer.forward(torch.from_numpy(make_workload("fc1").X.astype(np.float32)).to(torch.bfloat16)
+                               .to(dev))
+        X2 = torch.nn.functional.gelu(Y1.float(), approximate="tanh").to(torch.bfloat16)
+        wl.X = X2.double().cpu().numpy()
+        del Y1, X2
+    data = calibrate(wl.X, wl.W, wl.r, wl.alpha, bias=wl.bias, lora_A=wl.lora_A, lora_B=wl.lora_B)
+    lo, hi = rows if rows is not None else (0, wl.M)
+    M = hi - lo
+    K, N, r = wl.K, wl.N, data.r
+    layers = [SVDQLinear(data, device=dev) for _ in range(N_COPIES)]
+    X0 = torch.from_numpy(wl.X[lo:hi].astype(np.float32)).to(torch.bfloat16)
+    s = {"wl": wl, "data": data, "M": M, "K": K, "N": N, "r": r, "layers": layers, "X0": X0,
+         "Xs": [X0.to(dev) for _ in range(N_COPIES)],
+         "Ys": [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(N_COPIES)],
+         "LA": [torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev) if r else None for _ in range(N_COPIES)],
+         "ws": [C.new_workspace(M, K, r, dev) for _ in range(N_COPIES)]}
+    for L in layers:
+        L.act_buffers(M)
+    torch.cuda.synchronize()
+    return s
+
+
+def layer_fns(s):
+    from w4a4_rank_absorbed_b200 import svdq as C
+    M, K, N, r = s["M"], s["K"], s["N"], s["r"]
+    layers, Xs, Ys, LA, ws = s["layers"], s["Xs"], s["Ys"], s["LA"], s["ws"]
+
+    def quantize(i):
+        return layers[i % N_COPIES].quantize(Xs[i % N_COPIES])
+
+    def gemm(i):
+        L = layers[i % N_COPIES]
+        Xq, SFx, LAs = L.act_buffers(M)
+        L.gemm(Xq, SFx, LAs, Ys[i % N_COPIES])
+
+    def step(i):
+        quantize(i)
+        gemm(i)
+
+    def plain_qa(i):
+        L = layers[i % N_COPIES]
+        Xq, SFx, _ = L.act_buffers(M)
+        C.svdq_quantize_act(Xs[i % N_COPIES], M, K, L.inv_s, L.gs_x, None, 0, 1.0, Xq, SFx, None)
+
+    def plain_ln(i):
+        L = layers[i % N_COPIES]
+        Xq, SFx, _ = L.act_buffers(M)
+        C.svdq_linear(Xq, SFx, L.gs_x, L.Wq, L.SFw, L.gs_w, None, None, 0, L.bias, Ys[i % N_COPIES], 0, M, N, K)
+
+    def plain(i):
+        plain_qa(i)
+        plain_ln(i)
+
+    def down(i):
+        L = layers[i % N_COPIES]
+        C.svdq_lowrank_down(Xs[i % N_COPIES], M, K, L.L1fT, r, 1.0, LA[i % N_COPIES], ws[i % N_COPIES])
+
+    def up(i):
+        L = layers[i % N_COPIES]
+        C.svdq_lowrank_up(LA[i % N_COPIES], L.L2p, r, 1.0, Ys[i % N_COPIES], 0, M, N)
+
+    def unfused(i):
+        plain_qa(i)
+        down(i)
+        plain_ln(i)
+        up(i)
+
+    return {"quantize": quantize, "gemm": gemm, "step": step, "plain": plain, "plain_qa": plain_qa,
+            "plain_ln": plain_ln, "down": down, "up": up, "unfused": unfused}
+
+
+def measure_set(s, timer, dev, flush_buf):
+    """Every per-launch distribution of one workload, from the same graph protocol."""
+    import torch
+    fns = layer_fns(s)
+    r = s["r"]
+    for i in range(N_COPIES):          # eager once: lazily created state outside the graphs
+        fns["unfused"](i) if r else fns["plain"](i)
+        fns["step"](i)
+    torch.cuda.synchronize()
+    out = {}
+    for key in ("step", "quantize", "gemm", "plain", "plain_qa", "plain_ln"):
+        out[key] = timer.per_launch(fns[key])
+    if r:
+        for key in ("unfused", "down", "up"):
+            out[key] = timer.per_launch(fns[key])
+    # L2-warm: one layer copy over and over (its inputs, codes and weight stay in the L2 between steps).
+    out["step_l2_warm"] = timer.per_launch(lambda i: fns["step"](0))
+    # L2-flushed: a 256 MB write before every step on one copy, minus the same writes alone.
+    flush = lambda i: flush_buf.fill_(i & 0xFF)                       # noqa: E731
+    both = timer.per_launch(lambda i: (flush(i), fns["step"](0)))
+    alone = timer.per_launch(flush)
+    out["step_l2_flushed"] = [b - a for b, a in zip(both, alone)]
+    return out
+
+
+def workload_report(s, dist_ms, hbm_peak, fp4_peak):
+    M, K, N, r = s["M"], s["K"], s["N"], s["r"]
+    st = {k: stats(v) for k, v in dist_ms.items()}
+    med = {k: v["median"] for k, v in st.items()}
+    ln_fl = linear_flops(M, K, N, r)
+    qa_b = quantize_bytes(M, K, r)
+    rep = {
+        "M": M, "K": K, "N": N, "r": r,
+        "ms": st,
+        "tflops_step": layer_flops(M, K, N, r) / (med["step"] * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "svdq_linear (k_linear)",
+                     "achieved": ln_fl / (med["gemm"] * 1e-3) / 1e12, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": ln_fl / (med["gemm"] * 1e-3) / 1e12 / fp4_peak,
+                     "flops_per_launch": ln_fl, "ms_per_launch": med["gemm"]},
+        "svdq_quantize_act": {"ms": med["quantize"], "GB_per_s": qa_b / (med["quantize"] * 1e-3) / 1e9,
+                              "frac": qa_b / (med["quantize"] * 1e-3) / 1e9 / hbm_peak,
+                              "algorithmic_bytes": qa_b},
+        "lowrank_branch": {"fused_overhead": med["step"] / med["plain"] - 1.0, "gate_fused_overhead": 0.15},
+    }
+    if r:
+        extra = unfused_extra_bytes(M, K, N, r)
+        rep["lowrank_branch"].update({
+            "unfused_overhead": med["unfused"] / med["plain"] - 1.0,
+            "unfused": "in-house: kernel 2 at r = 0, svdq_lowrank_down (re-reads X), kernel 3 at r = 0, "
+                       "svdq_lowrank_up (reads and rewrites Y)",
+            "unfused_extra_bytes": extra,
+            "down_GB_per_s": (2.0 * M * K + 2.0 * M * r) / (med["down"] * 1e-3) / 1e9,
+            "up_GB_per_s": (4.0 * M * N + 4.0 * M * r) / (med["up"] * 1e-3) / 1e9})
+    return rep
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -247,158 +487,132 @@ def run_ours(args):
 
     from w4a4_rank_absorbed_b200 import build
     build.build()
-    from w4a4_rank_absorbed_b200.calib import calibrate
-    from w4a4_rank_absorbed_b200.layer import SVDQLinear
+    from w4a4_rank_absorbed_b200 import svdq as C
     from w4a4_rank_absorbed_b200.synth import make_workload
 
-    wl = make_workload(args.workload, seed_offset=0)
-    data = calibrate(wl.X, wl.W, wl.r, wl.alpha, bias=wl.bias, lora_A=wl.lora_A, lora_B=wl.lora_B)
-    M, K, N, r = wl.M, wl.K, wl.N, data.r
-    layers = [SVDQLinear(data, device=dev) for _ in range(N_COPIES)]
-    X0 = torch.from_numpy(wl.X.astype(np.float32)).to(torch.bfloat16)
-    Xs = [X0.to(dev) for _ in range(N_COPIES)]
-    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(N_COPIES)]
-    for L in layers:
-        L.act_buffers(M)
-    torch.cuda.synchronize()
+    bf16_peak, hbm_peak, peak_kind = peaks()
+    fp4_peak = bf16_peak * FP4_OVER_BF16
+    timer = Timer(torch, dev)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def quantize(i):
-        return layers[i % N_COPIES].quantize(Xs[i % N_COPIES])
+    wl0 = make_workload(args.workload)
+    rows = row_block(wl0.M, rank, world) if (args.strong and world > 1) else None
+    del wl0
+    fc1_layer = None
+    names = [args.workload] + [w for w in (args.extra.split(",") if args.extra else []) if w and w != args.workload]
+    if "fc2" in names and "fc1" not in names:
+        names.insert(names.index("fc2"), "fc1")
+    reports, clk_all, head = {}, [], None
+    for name in names:
+        s = build_layer_set(name, dev, rows=rows if name == args.workload else None, fc1_layer=fc1_layer)
+        clocks = ClockSampler(local)
+        clocks.start()
+        time.sleep(0.2)
+        d = measure_set(s, timer, dev, flush_buf)
+        if name == args.workload:
+            head = headline_steps(s, args, timer, dev, world, dist)
+        clk_all.append(clocks.stop())
+        st, site = C.svdq_get_device_error()
+        if st != 0:
+            raise SystemExit(f"device error {st} at {site:#x}")
+        keys = sorted(d)
+        maxed = max_over_ranks([x for k in keys for x in d[k]], device=dev)
+        pos = 0
+        for k in keys:
+            d[k], pos = maxed[pos:pos + len(d[k])], pos + len(d[k])
+        reports[name] = workload_report(s, d, hbm_peak, fp4_peak)
+        if name == args.workload:
+            e2e = None if args.no_e2e else e2e_leg(s, args, dev, world, dist)
+            head_set = {"M": s["M"], "K": s["K"], "N": s["N"], "r": s["r"], "wl": s["wl"], "data": s["data"]}
+        if name == "fc1":
+            fc1_layer = s["layers"][0]
+            s["layers"] = s["layers"][:1]
+        del s
+        torch.cuda.empty_cache()
+    # Kernel 1 (offline weight packing, HBM-bound) on the headline layer: one packing of its residual R.
+    pack = pack_leg(head_set["data"], dev, timer)
+    del fc1_layer
 
-    def gemm(i):
-        L = layers[i % N_COPIES]
-        Xq, SFx, LAs = L.act_buffers(M)
-        L.gemm(Xq, SFx, LAs, Ys[i % N_COPIES])
+    M, K, N, r = head_set["M"], head_set["K"], head_set["N"], head_set["r"]
+    ms = max_over_ranks([head], device=dev)[0]
+    fl = layer_flops(M, K, N, r)
+    value = job_throughput(fl, world, ms)
+    hr = reports[args.workload]
+    clk = ClockSampler.summarize([]) if not clk_all else {
+        "sm_mhz": statistics.median([c["sm_mhz"] for c in clk_all if c["sm_mhz"] is not None] or [0]),
+        "sm_max_mhz": max((c["sm_max_mhz"] or 0) for c in clk_all),
+        "reasons": sorted({x for c in clk_all for x in c["reasons"]}),
+        "samples": sum(c.get("samples", 0) for c in clk_all)}
+    roof = dict(hr["roofline"])
+    roof.update({"traffic": linear_traffic(args.workload),
+                 "peak_source": f"{peak_kind} bf16 {bf16_peak:.1f} TFLOP/s x {FP4_OVER_BF16:.0f} (nominal "
+                                f"NVFP4:bf16 dense ratio), burst: kernels timed in graphs of {GRAPH_LAUNCHES}",
+                 "timing": f"median over {GRAPH_REPLAYS} replays of a graph of {GRAPH_LAUNCHES} launches"})
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong" if (args.strong and world > 1) else "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded PCG64, random-init layer)",
+        "config": workload_config(head_set["wl"], args),
+        "pct_of_nvfp4_peak": 100.0 * (value / world) / fp4_peak,
+        "roofline": roof,
+        "kernels": {"svdq_quantize_act": dict(hr["svdq_quantize_act"], hbm_peak_GB_per_s=hbm_peak),
+                    "svdq_linear": {"ms": hr["roofline"]["ms_per_launch"], "TFLOP_per_s": hr["roofline"]["achieved"]},
+                    "svdq_pack_weight": pack},
+        "lowrank_branch": hr["lowrank_branch"],
+        "l2": {"rotating_ms": hr["ms"]["step"], "warm_ms": hr["ms"]["step_l2_warm"],
+               "flushed_ms": hr["ms"]["step_l2_flushed"]},
+        "workloads": {k: v for k, v in reports.items()},
+        "protocol": f"every 'ms' distribution: a CUDA graph of {GRAPH_LAUNCHES} launches (or steps) replayed "
+                    f"{GRAPH_REPLAYS} times, each replay timed with CUDA events, max over ranks; median, p10, p90 "
+                    f"per launch; the headline ms_per_step is one replay of a graph of exactly --steps steps",
+        "clocks": clk,
+        "gpu_launches": 2 * args.steps,
+    }
+    if e2e is not None:
+        out["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wl = make_workload(args.workload)
+        out["cpu_baseline"] = cpu_baseline(wl, min(args.cpu_sample_rows or wl.M, wl.M))
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
 
+
+def headline_steps(s, args, timer, dev, world, dist):
+    """The contract's timed region: W untimed warm-up steps, then exactly K steps in one graph replay,
+    bracketed by a barrier and a device synchronisation on both sides."""
+    import torch
+    fns = layer_fns(s)
     for i in range(args.warmup):
-        quantize(i)
-        gemm(i)
+        fns["step"](i)
     torch.cuda.synchronize()
-
-    from w4a4_rank_absorbed_b200 import svdq as C
-
-    # The K timed steps are captured in one CUDA graph (step i: kernel 2 then kernel 3 on layer
-    # copy i % N_COPIES) and the timed region is one replay of it: device time, without the
-    # Python/ctypes launch overhead or the gaps between separately launched graphs.  The
-    # per-kernel averages come from two more graphs holding only kernel 2 or only kernel 3
-    # launches over the same copies, timed the same way right after.
-    def capture(fn, n):
-        g = torch.cuda.CUDAGraph()
-        cap = torch.cuda.Stream(device=dev)
-        cap.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(cap):
-            # thread_local: under torchrun the process group's watchdog thread queries CUDA events
-            # while we capture; the default (global) mode would invalidate the capture.
-            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
-                for i in range(n):
-                    fn(i)
-        torch.cuda.current_stream().wait_stream(cap)
-        return g
-
-    def step(i):
-        quantize(i)
-        gemm(i)
-
-    n_kernel = 4 * N_COPIES
-    g_steps = capture(step, args.steps)
-    g_qa = capture(quantize, n_kernel)
-    g_ln = capture(gemm, n_kernel)
-    for g in (g_steps, g_qa, g_ln):        # warm replays, untimed
-        g.replay()
+    g = timer.capture(fns["step"], args.steps)
+    g.replay()
     torch.cuda.synchronize()
-
-    def timed(g):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1)
-
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ms = timed(g_steps) / args.steps
+    ms = timer.replay_ms(g) / args.steps
     if world > 1:
         dist.barrier()
-    t_qa = timed(g_qa) / n_kernel
-    t_ln = timed(g_ln) / n_kernel
-    clk = clocks.stop()
-    st, site = C.svdq_get_device_error()
-    if st != 0:
-        raise SystemExit(f"device error {st} at {site:#x}")
-    # The same layer without its low-rank branch (kernel 2 with r = 0, kernel 3 with r = 0) and
-    # with the branch unfused (down-projection X L1f and up-projection Y += LA L2 as separate
-    # cuBLAS calls that re-read X and re-read and re-write Y): the cost of the branch, fused and not.
-
-    def plain(i):
-        L = layers[i % N_COPIES]
-        Xq, SFx, _ = L.act_buffers(M)
-        C.svdq_quantize_act(Xs[i % N_COPIES], M, K, L.inv_s, L.gs_x, None, 0, 1.0, Xq, SFx, None)
-        C.svdq_linear(Xq, SFx, L.gs_x, L.Wq, L.SFw, L.gs_w, None, None, 0, L.bias, Ys[i % N_COPIES], 0, M, N, K)
-
-    lr = []
-    for L in layers:
-        if r:
-            lr.append((L.L1fT.t().contiguous(), L.L2p[:, :r].t().contiguous(),
-                       torch.empty((M, r), dtype=torch.bfloat16, device=dev)))
-
-    def unfused(i):
-        plain(i)
-        if r:
-            L1f, L2b, LA = lr[i % N_COPIES]
-            torch.matmul(Xs[i % N_COPIES], L1f, out=LA)
-            Ys[i % N_COPIES].addmm_(LA, L2b)
-
-    for i in range(N_COPIES):              # eager first: creates the cuBLAS handle and workspace
-        unfused(i)
     torch.cuda.synchronize()
-    g_plain = capture(plain, n_kernel)
-    g_unf = capture(unfused, n_kernel)
-    g_plain.replay()
-    g_unf.replay()
-    torch.cuda.synchronize()
-    t_plain = timed(g_plain) / n_kernel
-    t_unf = timed(g_unf) / n_kernel
-    # L2-warm step: the same two kernels on one layer copy over and over (its inputs, codes and
-    # weight stay in the 126 MB L2 between steps).
-    g_warm = capture(lambda i: step(0), n_kernel)
-    g_warm.replay()
-    torch.cuda.synchronize()
-    t_warm = timed(g_warm) / n_kernel
-    # Kernel 1 (offline weight packing, HBM-bound): one packing of the layer's residual R.
-    L0 = layers[0]
-    R_dev = data.R.to(dev, torch.float32).contiguous()
-    L2b_dev = L0.L2p[:, :r].t().contiguous() if r else None
-    Wq_t, SFw_t = torch.empty_like(L0.Wq), torch.empty_like(L0.SFw)
-    gsw_t = torch.empty(1, dtype=torch.float32, device=dev)
-    L2p_t = torch.empty_like(L0.L2p) if r else None
+    del g
+    return ms
 
-    def pack(i):
-        C.svdq_pack_weight(R_dev, L2b_dev, K, N, r, Wq_t, SFw_t, gsw_t, L2p_t)
 
-    pack(0)
-    torch.cuda.synchronize()
-    g_pack = capture(pack, 4)
-    g_pack.replay()
-    torch.cuda.synchronize()
-    t_pack = timed(g_pack) / 4
-    del R_dev
-    ms, t_qa, t_ln, t_plain, t_unf, t_warm, t_pack = max_over_ranks(
-        [ms, t_qa, t_ln, t_plain, t_unf, t_warm, t_pack], device=dev)
-    del g_steps, g_qa, g_ln, g_plain, g_unf, g_warm, g_pack
-
-    # End to end through the public API with host buffers: every step copies its X in from pinned
-    # host memory and its Y out to pinned host memory inside the timed region.  The layer's
-    # streamed call overlaps step i's kernels with step i+1's copy in and step i-1's copy out.
-    Xh = X0.pin_memory()
+def e2e_leg(s, args, dev, world, dist):
+    """End to end through the public API with host buffers: every step copies its X in from pinned host
+    memory and its Y out to pinned host memory inside the timed region (the layer's streamed call overlaps
+    step i's kernels with step i+1's copy in and step i-1's copy out)."""
+    import torch
+    M, K, N, r = s["M"], s["K"], s["N"], s["r"]
+    Xh = s["X0"].pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
     Yhs = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    X_devs, Y_devs = Xs[:2], Ys[:2]
-    L0 = layers[0]
+    L0 = s["layers"][0]
+    X_devs, Y_devs = s["Xs"][:2], s["Ys"][:2]
     L0.forward_host_stream([Xh] * 2, Yhs, X_devs, Y_devs)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -410,51 +624,32 @@ def run_ours(args):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], device=dev)[0]
-
     fl = layer_flops(M, K, N, r)
-    value = job_throughput(fl, world, ms)
-    bf16_peak, hbm_peak, peak_kind = peaks()
-    fp4_peak = bf16_peak * FP4_OVER_BF16
-    lin_flops = 2.0 * M * N * K + 2.0 * M * N * r
-    lin_tf = lin_flops / (t_ln * 1e-3) / 1e12
-    qa_bytes = 2.0 * M * K + M * K / 2 + M * K / 16 + 2.0 * M * r
-    pack_bytes = 4.0 * K * N + K * N / 2 + K * N / 16 + 2.0 * r * N + 4.0 * N * r
-    qa_gbs = qa_bytes / (t_qa * 1e-3) / 1e9
+    return {"value": job_throughput(fl, world, e2e_ms), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 2), "ms_per_step": e2e_ms}
 
-    out = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded PCG64, random-init layer)",
-        "config": workload_config(wl),
-        "pct_of_nvfp4_peak": 100.0 * (value / world) / fp4_peak,
-        "roofline": {"bound": "tensor", "kernel": "svdq_linear (k_linear)", "achieved": lin_tf, "peak": fp4_peak,
-                     "unit": "TFLOP/s", "frac": lin_tf / fp4_peak, "traffic": linear_traffic(args.workload),
-                     "peak_source": f"{peak_kind} bf16 {bf16_peak:.1f} TFLOP/s x {FP4_OVER_BF16:.0f} (nominal "
-                                    f"NVFP4:bf16 dense ratio)",
-                     "flops_per_launch": lin_flops, "ms_per_launch": t_ln},
-        "kernels": {"svdq_quantize_act": {"ms": t_qa, "GB_per_s": qa_gbs, "hbm_peak_GB_per_s": hbm_peak,
-                                          "frac": qa_gbs / hbm_peak, "algorithmic_bytes": qa_bytes},
-                    "svdq_linear": {"ms": t_ln, "TFLOP_per_s": lin_tf},
-                    "svdq_pack_weight": {"ms": t_pack, "GB_per_s": pack_bytes / (t_pack * 1e-3) / 1e9,
-                                         "algorithmic_bytes": pack_bytes,
-                                         "note": "offline, once per layer; not in the step"}},
-        "l2_warm_ms_per_step": t_warm,
-        "lowrank_branch": {"fused_ms_per_step": ms, "without_branch_ms_per_step": t_plain,
-                           "unfused_ms_per_step": t_unf, "fused_overhead": ms / t_plain - 1.0,
-                           "unfused_overhead": t_unf / t_plain - 1.0, "gate_fused_overhead": 0.15,
-                           "unfused": "kernel 2 and 3 at r = 0, then X L1f and Y += LA L2 as cuBLAS bf16 calls"},
-        "clocks": clk,
-        "e2e": {"value": job_throughput(fl, world, e2e_ms), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 2), "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = min(args.cpu_sample_rows or M, M)       # default: every row of the step (a few s of CPU)
-        out["cpu_baseline"] = cpu_baseline(wl, rows)
-    if rank == 0:
-        print(json.dumps(out), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+
+def pack_leg(data, dev, timer):
+    import torch
+
+    from w4a4_rank_absorbed_b200 import svdq as C
+    K, N, r = data.K, data.N, data.r
+    R_dev = data.R.to(dev, torch.float32).contiguous()
+    L2b_dev = data.L2b.to(dev).contiguous() if r else None
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    SFw = torch.empty(C.svdq_sf_bytes(N, K), dtype=torch.uint8, device=dev)
+    gsw = torch.empty(1, dtype=torch.float32, device=dev)
+    L2p = torch.empty((N, r), dtype=torch.bfloat16, device=dev) if r else None
+
+    def pack(i):
+        C.svdq_pack_weight(R_dev, L2b_dev, K, N, r, Wq, SFw, gsw, L2p, sync=False)
+
+    pack(0)
+    torch.cuda.synchronize()
+    st = stats(timer.per_launch(pack, n=4, reps=10))
+    pack_bytes = 4.0 * K * N + K * N / 2 + K * N / 16 + 2.0 * r * N + 2.0 * N * r
+    return {"ms": st["median"], "GB_per_s": pack_bytes / (st["median"] * 1e-3) / 1e9, "algorithmic_bytes": pack_bytes,
+            "note": "offline, once per layer; not in the step"}
 
 
 def main():

@@ -34,7 +34,8 @@
  *
  * Conventions for every call:
  *   - Pointers are device pointers unless stated; the caller owns and
- *     allocates every buffer; the library allocates no device memory.
+ *     allocates every buffer, workspaces included; the library allocates no
+ *     device memory.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  Argument errors are returned before any launch;
  *     a launch failure returns SVDQ_ERR_CUDA.  Kernel-side faults that do not
@@ -100,16 +101,30 @@ SVDQ_API size_t svdq_sf_bytes(int64_t rows, int64_t K);
  *   gs_w [out] float32 (one device float): the weight global scale,
  *              amax(|R|) / 2688; also used as the amax accumulator while the
  *              call runs, so it must not alias anything else.
- *   L2p  [out] bf16, N x 2r row-major: row n = [L2b[:, n] , L2b[:, n]], the
- *              up-projection laid out K-major for the GEMM, doubled so that
- *              the high and low halves of LAs (see svdq_quantize_act) meet
- *              the same factor (NULL when r == 0).
- * Four launches (zero, amax, scale, encode).  The caller reads gs_w back to
- * form lr_scale for svdq_quantize_act.
+ *   gs_w_host [out] HOST float or NULL.  When given, the call copies gs_w to
+ *              it and synchronises `stream` before returning (the caller
+ *              needs the value to form lr_scale for svdq_quantize_act and the
+ *              scale argument of svdq_linear).  When NULL the call is
+ *              asynchronous like the others.
+ *   L2p  [out] bf16, N x r row-major: row n = L2b[:, n], the up-projection
+ *              laid out K-major for the GEMM (NULL when r == 0).
+ * Five launches (zero, amax, scale, encode, L2 layout).
  */
 SVDQ_API svdq_status svdq_pack_weight(const float* R, const uint16_t* L2b, int64_t K, int64_t N, int r,
-                             uint8_t* Wq, uint8_t* SFw, float* gs_w, uint16_t* L2p,
+                             uint8_t* Wq, uint8_t* SFw, float* gs_w, float* gs_w_host, uint16_t* L2p,
                              svdq_stream_t stream);
+
+/*
+ * svdq_dequant_weight -- the value of a packed weight, Q(R), for the offline
+ * refinement of the decomposition (SVDQuant review, §4.2: R is optimized
+ * repeatedly to minimize the quantization error, which needs Q(R) itself).
+ *
+ *   Wq, SFw, gs_w [in] from svdq_pack_weight (gs_w the device float).
+ *   Rq   [out] float32, K x N row-major:
+ *              Rq[k, n] = f32(e2m1(code) * f32(dec(sb) * gs_w)), sign from the code.
+ */
+SVDQ_API svdq_status svdq_dequant_weight(const uint8_t* Wq, const uint8_t* SFw, const float* gs_w, int64_t K,
+                                int64_t N, float* Rq, svdq_stream_t stream);
 
 /*
  * svdq_quantize_act -- activation kernel with the fused down-projection
@@ -128,13 +143,33 @@ SVDQ_API svdq_status svdq_pack_weight(const float* R, const uint16_t* L2b, int64
  *                  one accumulator and scale once by gs_x * gs_w.
  *   Xq       [out] uint8, M x K/2: E2M1 codes of X_hat.
  *   SFx      [out] uint8, svdq_sf_bytes(M, K): UE4M3 scales, MMA scale order.
- *   LAs      [out] bf16, M x 2r: row m = [hi(v) | lo(v)] with
+ *   workspace [in/out] device memory of at least
+ *                  svdq_quantize_act_workspace_bytes(M, K, r) bytes (NULL and 0
+ *                  when r == 0).  When a row block's 128 rows are too few to
+ *                  fill the GPU, up to 8 CTAs share the block's K axis and add
+ *                  their partial down-projections here; the first bytes are one
+ *                  counter per row block that the kernel leaves at 0.  Zero the
+ *                  whole workspace once after allocating it (and again after a
+ *                  call that reported SVDQ_ERR_TIMEOUT); calls on streams that
+ *                  may overlap need workspaces of their own.
+ *   LAs      [out] bf16, M x 2r: the hi/lo pair of
  *                  v = f32(lr_scale * (X L1f)[m, :]) (fp32 accumulation),
- *                  hi = bf16_rne(v), lo = bf16_rne(v - hi).  NULL when r == 0.
+ *                  hi = bf16_rne(v), lo = bf16_rne(v - hi), interleaved by 16
+ *                  columns: LAs[m, 32j + t] = hi(v[16j + t]) and
+ *                  LAs[m, 32j + 16 + t] = lo(v[16j + t]) for t < 16 (the order
+ *                  svdq_linear's rank stage reads).  NULL when r == 0.
+ * Launched as a programmatic dependent of the previous kernel on the stream
+ * (its set-up overlaps that kernel's tail; it reads X only after that kernel
+ * has finished).
  */
 SVDQ_API svdq_status svdq_quantize_act(const uint16_t* X, int64_t M, int64_t K, const float* inv_s,
                               float gs_x, const uint16_t* L1fT, int r, float lr_scale,
-                              uint8_t* Xq, uint8_t* SFx, uint16_t* LAs, svdq_stream_t stream);
+                              uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
+                              void* workspace, size_t workspace_bytes, svdq_stream_t stream);
+
+/* Bytes of the workspace svdq_quantize_act and svdq_lowrank_down need for M rows of K columns at
+ * rank r (0 when r == 0; 0 for a shape the calls reject).  Independent of the device. */
+SVDQ_API size_t svdq_quantize_act_workspace_bytes(int64_t M, int64_t K, int r);
 
 /*
  * svdq_linear -- block-scaled NVFP4 GEMM on the tcgen05 tensor cores with the
@@ -149,13 +184,50 @@ SVDQ_API svdq_status svdq_quantize_act(const uint16_t* X, int64_t M, int64_t K, 
  *   LAs, L2p    [in] may be NULL when r == 0 (plain NVFP4 GEMM).
  *   bias        [in] bf16, N, or NULL.
  *   Y           [out] M x N row-major: bf16 when y_fp32 == 0, float32 when 1.
- * Persistent, warp-specialised kernel: one CTA per SM, 128 x 256 output tiles.
+ * Persistent, warp-specialised kernel: one CTA per SM, 128 x 256 output tiles,
+ * launched as a programmatic dependent of the previous kernel on the stream
+ * (set-up overlaps that kernel's tail; inputs are read and Y written only
+ * after it has finished).
  */
 SVDQ_API svdq_status svdq_linear(const uint8_t* Xq, const uint8_t* SFx, float gs_x,
                         const uint8_t* Wq, const uint8_t* SFw, float gs_w,
                         const uint16_t* LAs, const uint16_t* L2p, int r,
                         const uint16_t* bias, void* Y, int y_fp32,
                         int64_t M, int64_t N, int64_t K, svdq_stream_t stream);
+
+/*
+ * svdq_lowrank_down -- the low-rank down-projection as a kernel of its own: the
+ * unfused form of the branch (SVDQuant review, §4.3: without fusion the branch
+ * re-reads the 16-bit activations from memory, which is what the fused
+ * svdq_quantize_act avoids).  Kept to measure what the fusion buys.
+ *
+ *   X, M, K, L1fT, r, lr_scale, workspace: as in svdq_quantize_act (r >= 16).
+ *   LAs [out] bf16, M x 2r, the same layout and values as svdq_quantize_act's
+ *       LAs for the same inputs (the two kernels share the down-projection
+ *       code; this one skips the quantization).
+ */
+SVDQ_API svdq_status svdq_lowrank_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* L1fT, int r,
+                              float lr_scale, uint16_t* LAs, void* workspace, size_t workspace_bytes,
+                              svdq_stream_t stream);
+
+/*
+ * svdq_lowrank_up -- the low-rank up-projection as a kernel of its own, adding
+ * into an existing output (the unfused form of the branch, SVDQuant review,
+ * §4.3: without fusion the branch reads and rewrites the output):
+ *
+ *   Y[m, n] = round(gs * sum_t (hi + lo)(LAs)[m, t] * L2p[n, t] + Y[m, n])
+ *
+ *   LAs  [in]  bf16, M x 2r, the layout of svdq_quantize_act / svdq_lowrank_down.
+ *   L2p  [in]  bf16, N x r, from svdq_pack_weight (r >= 16).
+ *   gs   [in]  host float: the scale of the product (gs_x * gs_w when LAs was
+ *              pre-scaled by lr_scale = 1 / (gs_x * gs_w); 1 when it was not).
+ *   Y    [in/out] M x N row-major, bf16 (y_fp32 = 0) or float32 (y_fp32 = 1),
+ *              read and rewritten; rounded once to its own type.
+ * The tcgen05 GEMM kernel of svdq_linear with no 4-bit tiles, only the rank
+ * tiles, and an epilogue that reads Y instead of the bias.
+ */
+SVDQ_API svdq_status svdq_lowrank_up(const uint16_t* LAs, const uint16_t* L2p, int r, float gs, void* Y, int y_fp32,
+                            int64_t M, int64_t N, svdq_stream_t stream);
 
 /*
  * svdq_get_device_error -- synchronises `stream`, then reads and clears the
@@ -169,12 +241,8 @@ SVDQ_API svdq_status svdq_get_device_error(svdq_stream_t stream, int* site);
 /*
  * svdq_linear_debug -- svdq_linear with test hooks, for the fault-path tests.
  *   debug_flags bit 0: the load warp issues no loads, so the MMA warp's first
- *                      wait can never complete and must run out.
- *               bit 1: use the single-CTA kernel (128 x 256 tiles) whatever M is.
- *               bit 2: use the CTA-pair kernel (256 x 256 tiles) whatever M is.
- *   (svdq_linear itself uses the single-CTA kernel; the CTA-pair kernel gives the same
- *   results up to the fp32 accumulation order and is kept for comparison.  Setting both
- *   bits 1 and 2 is SVDQ_ERR_INVALID_ARG.)
+ *                      wait can never complete and must run out.  Any other
+ *                      bit is SVDQ_ERR_INVALID_ARG.
  *   timeout_ns: bound of every barrier wait (0 = the default of 2 s).
  * Otherwise identical to svdq_linear.
  */

@@ -88,13 +88,17 @@ def activation_global_scale(X, inv_s) -> np.float32:
 
 
 def decompose(X, W, r: int, alpha: float = 0.5, lora_A: Optional[np.ndarray] = None,
-              lora_B: Optional[np.ndarray] = None, X_cal=None) -> Decomposition:
+              lora_B: Optional[np.ndarray] = None, X_cal=None, refine_iters: int = 0) -> Decomposition:
+    """refine_iters > 0: the low-rank split is refined against the 4-bit residual (oracle.refine)."""
     X = np.asarray(X, dtype=np.float64)
     W = np.asarray(W, dtype=np.float64)
     Xc = X if X_cal is None else np.asarray(X_cal, dtype=np.float64)
     s = smoothing_factors(Xc, W, alpha)
     W_hat = s[:, None] * W
     L1, L2, R, S = low_rank_split(W_hat, r)
+    if refine_iters > 0:
+        from .refine import refine
+        L1, L2, R, _ = refine(W_hat, r, refine_iters)
     if lora_A is not None:
         L1 = np.concatenate([L1, s[:, None] * lora_A], axis=1)
         L2 = np.concatenate([L2, lora_B], axis=0)

@@ -39,6 +39,15 @@ def test_status_strings_and_sizes(lib):
     assert svdq.svdq_sf_bytes(10, 100) == 0
 
 
+def test_workspace_size_query(lib):
+    # ticket words (one per 128-row block, padded to 256 bytes), then up to 8 partial sums of M x r floats
+    assert svdq.svdq_quantize_act_workspace_bytes(4608, 3072, 0) == 0
+    assert svdq.svdq_quantize_act_workspace_bytes(4608, 3072, 32) == 256 + 8 * 4608 * 32 * 4
+    assert svdq.svdq_quantize_act_workspace_bytes(200, 512, 16) == 256 + 8 * 256 * 16 * 4
+    assert svdq.svdq_quantize_act_workspace_bytes(100, 96, 16) == 0        # K % 64: rejected shape
+    assert svdq.svdq_quantize_act_workspace_bytes(100, 128, 24) == 0       # r % 16
+
+
 def _linear(lib, **kw):
     a = dict(Xq=16, SFx=16, gs_x=1.0, Wq=16, SFw=16, gs_w=1.0, LAs=16, L2p=16, r=32, bias=None, Y=16,
              y_fp32=0, M=128, N=256, K=256, stream=None)
@@ -60,13 +69,23 @@ def test_argument_errors_before_any_launch(lib):
     assert _linear(lib, y_fp32=2) == svdq.SVDQ_ERR_INVALID_ARG
     assert _linear(lib, Y=24) == svdq.SVDQ_ERR_MISALIGNED
     assert _linear(lib, bias=8) == svdq.SVDQ_ERR_MISALIGNED
-    assert lib.svdq_quantize_act(16, 64, 100, 16, 1.0, 16, 32, 1.0, 16, 16, 16, None) == \
+    ws = svdq.svdq_quantize_act_workspace_bytes(64, 128, 32)
+    assert lib.svdq_quantize_act(16, 64, 100, 16, 1.0, 16, 32, 1.0, 16, 16, 16, 16, ws, None) == \
         svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
-    assert lib.svdq_quantize_act(16, 64, 128, 16, 1.0, None, 32, 1.0, 16, 16, 16, None) == \
+    assert lib.svdq_quantize_act(16, 64, 128, 16, 1.0, None, 32, 1.0, 16, 16, 16, 16, ws, None) == \
         svdq.SVDQ_ERR_INVALID_ARG
-    assert lib.svdq_pack_weight(16, 16, 128, 40, 32, 16, 16, 16, 16, None) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
-    assert lib.svdq_pack_weight(4, 16, 128, 32, 32, 16, 16, 16, 16, None) == svdq.SVDQ_ERR_MISALIGNED
-    for flags in (8, 2 | 4):       # an unknown bit; both kernels forced at once
+    # a workspace missing or smaller than the query says
+    assert lib.svdq_quantize_act(16, 64, 128, 16, 1.0, 16, 32, 1.0, 16, 16, 16, None, 0, None) == \
+        svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_quantize_act(16, 64, 128, 16, 1.0, 16, 32, 1.0, 16, 16, 16, 16, ws - 1, None) == \
+        svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_lowrank_down(16, 64, 128, 16, 0, 1.0, 16, 16, ws, None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_lowrank_down(16, 64, 128, 16, 32, 1.0, 16, 8, ws, None) == svdq.SVDQ_ERR_MISALIGNED
+    assert lib.svdq_lowrank_up(16, 16, 0, 1.0, 16, 0, 64, 64, None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_lowrank_up(16, 16, 32, 1.0, 16, 0, 64, 40, None) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert lib.svdq_pack_weight(16, 16, 128, 40, 32, 16, 16, 16, None, 16, None) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert lib.svdq_pack_weight(4, 16, 128, 32, 32, 16, 16, 16, None, 16, None) == svdq.SVDQ_ERR_MISALIGNED
+    for flags in (2, 4, 8):        # only bit 0 is defined
         assert lib.svdq_linear_debug(16, 16, 1.0, 16, 16, 1.0, 16, 16, 32, None, 16, 0, 128, 256, 256, flags, 0,
                                      None) == svdq.SVDQ_ERR_INVALID_ARG
 

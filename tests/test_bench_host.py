@@ -41,3 +41,33 @@ def test_workload_config_names_the_workload_and_sizes():
     assert cfg["workload"].startswith("tiny")
     assert (cfg["M"], cfg["K"], cfg["N"], cfg["r"]) == (wl.M, wl.K, wl.N, wl.r_eff)
     assert "L2" in cfg["l2"] and "graph" in cfg["launch"]
+
+
+def test_row_blocks_partition_the_batch():
+    for M in (1, 7, 4608, 18432):
+        for world in (1, 2, 3, 8):
+            blocks = [bench.row_block(M, r, world) for r in range(world)]
+            assert blocks[0][0] == 0 and blocks[-1][1] == M
+            assert all(a[1] == b[0] for a, b in zip(blocks, blocks[1:]))
+            sizes = [hi - lo for lo, hi in blocks]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def test_stats_median_and_percentiles():
+    st = bench.stats([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert st["median"] == 3.0 and st["n"] == 5
+    assert 1.0 <= st["p10"] <= 2.0 and 4.0 <= st["p90"] <= 5.0
+
+
+def test_byte_counts():
+    M, K, N, r = 4608, 3072, 9216, 32
+    assert bench.quantize_bytes(M, K, r) == 2 * M * K + M * K / 2 + M * K / 16 + 2 * M * r
+    assert bench.linear_flops(M, K, N, r) == 2.0 * M * N * K + 2.0 * M * N * r
+    assert bench.unfused_extra_bytes(M, K, N, r) == 2.0 * M * K + 4.0 * M * N
+
+
+def test_clock_summary_flags_throttle_reasons():
+    rows = [["0", "1965", "1965", "900", "0x0", "Not Active", "Not Active", "Not Active", "Active"],
+            ["0", "1900", "1965", "950", "0x4", "Not Active", "Not Active", "Not Active", "Not Active"]]
+    got = bench.ClockSampler.summarize(rows)
+    assert got["sm_max_mhz"] == 1965.0 and got["reasons"] == ["sw_power_cap"] and got["samples"] == 2

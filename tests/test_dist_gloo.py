@@ -51,6 +51,50 @@ def test_max_over_ranks_and_weak_scaling_value():
         assert abs(val - 2000.0) < 1e-9
 
 
+def _shard_worker(rank, world, port, q):
+    # Strong scaling: one batch split into row blocks; every rank computes its block of a row-wise
+    # function and the blocks, gathered, must reassemble the whole batch's result in order.
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        M = 37
+        X = torch.arange(M * 3, dtype=torch.float64).reshape(M, 3)
+        lo, hi = bench.row_block(M, rank, world)
+        Y = (X[lo:hi] * 2.0 + 1.0).contiguous()
+        # blocks differ in size by at most one row: gather them padded to the largest, then trim
+        cap = max(b - a for a, b in (bench.row_block(M, r, world) for r in range(world)))
+        pad = torch.zeros((cap, 3), dtype=torch.float64)
+        pad[:hi - lo] = Y
+        parts = [torch.zeros((cap, 3), dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(parts, pad)
+        full = torch.cat([p[:b - a] for p, (a, b) in zip(parts, (bench.row_block(M, r, world)
+                                                                 for r in range(world)))])
+        q.put((rank, bool(torch.equal(full, X * 2.0 + 1.0)), (lo, hi)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_row_sharded_replicas_reassemble_the_batch():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(ok for _, ok, _ in out)
+    assert out[0][2] == (0, 18) and out[1][2] == (18, 37)
+
+
 def test_single_process_reduction_is_identity():
     sys.path.insert(0, ROOT)
     import bench

@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import (GpuLayer, OC, OD, OL, bf16_dev, bf16_host, check_las, check_y,
+from helpers import (GpuLayer, OC, OD, OL, bf16_dev, bf16_host, check_las, check_y, las_join,
                      mismatch_report, oracle_layer, oracle_storage, require_gpu, u8_host)
 from oracle.layout import sf_to_storage
 from w4a4_rank_absorbed_b200.synth import make_workload, small_case
@@ -35,8 +35,7 @@ def test_pack_weight_bitexact(K, N, r):
     _assert_bytes(g.Wq, ref["Wq"], "Wq")
     _assert_bytes(g.SFw, ref["SFw"], "SFw")
     if r:
-        want = np.concatenate([dec.L2b.T, dec.L2b.T], axis=1)
-        assert np.array_equal(bf16_host(g.L2p), want)
+        assert np.array_equal(bf16_host(g.L2p), dec.L2b.T)
     g.check_errors()
 
 
@@ -44,8 +43,9 @@ def test_pack_weight_bitexact(K, N, r):
                                    (130, 512, 48), (64, 256, 80), (64, 256, 128), (1, 64, 16), (160, 192, 96),
                                    (33, 320, 112)])
 def test_quantize_act_bitexact(M, K, r):
-    wl = small_case(M, K, 32, r, seed=M * 7 + K + r)
+    wl = small_case(M, K, 128, r, seed=M * 7 + K + r)
     dec = oracle_layer(wl, r)
+    assert dec.L1f.shape[1] == r       # N >= r, so the rank is not clamped
     g = GpuLayer(dec, wl.bias)
     Xq, SFx, LAs = g.quantize(bf16_dev(wl.X))
     qa = OL.quantize_act(wl.X, dec.inv_s, dec.gs_x, dec.L1f)
@@ -58,7 +58,8 @@ def test_quantize_act_bitexact(M, K, r):
 
 
 def _oracle_inputs_to_device(qa, pw, dec, lr_scale, r_expected):
-    """The oracle's codes/scales and a hi/lo split of its float64 low-rank product, as device buffers.
+    """The oracle's codes/scales and a hi/lo split of its float64 low-rank product (in the LAs layout:
+    interleaved by 16 columns), as device buffers.
 
     The buffers are sized by the decomposition's rank, which the launch must use: a kernel
     told a larger r would read past LAs and L2p.
@@ -73,8 +74,8 @@ def _oracle_inputs_to_device(qa, pw, dec, lr_scale, r_expected):
         v = torch.from_numpy((qa.LA * np.float64(lr_scale)).astype(np.float32))
         hi = v.to(torch.bfloat16)
         lo = (v - hi.float()).to(torch.bfloat16)
-        LAs = torch.cat([hi, lo], dim=1).contiguous().cuda()
-        L2p = bf16_dev(np.concatenate([dec.L2b.T, dec.L2b.T], axis=1))
+        LAs = bf16_dev(las_join(hi.double().numpy(), lo.double().numpy()))
+        L2p = bf16_dev(np.ascontiguousarray(dec.L2b.T))
     else:
         LAs = L2p = None
     return Xq, SFx, Wq, SFw, LAs, L2p
@@ -102,30 +103,6 @@ def test_linear_on_oracle_codes(M, N, K, r, use_bias, y_fp32):
     torch.cuda.synchronize()
     Y_or = OL.linear(qa, gs_x, pw, dec.L2b, wl.bias if use_bias else None)
     check_y(Y.float().cpu().numpy().astype(np.float64), Y_or, bf16=not y_fp32, what=f"Y {M}x{N}x{K} r={r}")
-    st, site = C.svdq_get_device_error()
-    assert st == 0, site
-
-
-@pytest.mark.parametrize("kernel", ["single", "pair"])
-@pytest.mark.parametrize("M,N,K,r", [(256, 512, 512, 32), (100, 272, 576, 16), (520, 1296, 1536, 128),
-                                     (384, 144, 64, 0), (1, 64, 128, 48)])
-def test_linear_single_and_pair_kernels(M, N, K, r, kernel):
-    # svdq_linear picks the CTA-pair kernel for M > 128; force each kernel on every shape.
-    from w4a4_rank_absorbed_b200 import svdq as C
-    wl = small_case(M, K, N, r, seed=5 * M + N + K)
-    dec = oracle_layer(wl, r)
-    pw = OL.pack_weight(dec.R32)
-    qa = OL.quantize_act(wl.X, dec.inv_s, dec.gs_x, dec.L1f)
-    gs_x, gs_w = np.float32(dec.gs_x), pw.gs_w
-    lr_scale = np.float32(1.0 / (np.float64(gs_x) * np.float64(gs_w)))
-    Xq, SFx, Wq, SFw, LAs, L2p = _oracle_inputs_to_device(qa, pw, dec, lr_scale, r)
-    bias = bf16_dev(wl.bias)
-    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
-    flag = 2 if kernel == "single" else 4
-    C.svdq_linear_debug(Xq, SFx, float(gs_x), Wq, SFw, float(gs_w), LAs, L2p, r, bias, Y, 1, M, N, K, flag, 0)
-    torch.cuda.synchronize()
-    Y_or = OL.linear(qa, gs_x, pw, dec.L2b, wl.bias)
-    check_y(Y.cpu().numpy().astype(np.float64), Y_or, bf16=False, what=f"{kernel} Y {M}x{N}x{K} r={r}")
     st, site = C.svdq_get_device_error()
     assert st == 0, site
 
@@ -230,4 +207,76 @@ def test_repeated_launches_are_identical_and_error_free():
             ref = cur
         else:
             assert cur == ref
+    g.check_errors()
+
+
+@pytest.mark.parametrize("M,K,r", [(256, 512, 32), (300, 1024, 64), (1152, 3072, 32), (37, 256, 16), (130, 512, 48)])
+def test_lowrank_down_equals_the_fused_down_projection(M, K, r):
+    # The separate down-projection (unfused pipeline) runs the fused kernel's MMA path without the
+    # quantization: its LAs must be bit-identical to the fused kernel's, and within the LA bound of the
+    # oracle's float64 product.
+    from w4a4_rank_absorbed_b200 import svdq as C
+    wl = small_case(M, K, 128, r, seed=3 * M + K + r)
+    dec = oracle_layer(wl, r)
+    assert dec.L1f.shape[1] == r, "the buffers are sized by the decomposition's rank"
+    g = GpuLayer(dec, wl.bias)
+    X = bf16_dev(wl.X)
+    _, _, LAs_fused = g.quantize(X)
+    LAs = torch.empty((M, 2 * r), dtype=torch.bfloat16, device="cuda")
+    C.svdq_lowrank_down(X, M, K, g.L1fT, r, float(g.lr_scale), LAs, C.new_workspace(M, K, r))
+    torch.cuda.synchronize()
+    assert torch.equal(LAs.view(torch.int16), LAs_fused.view(torch.int16))
+    check_las(LAs, wl.X, dec.L1f, g.lr_scale)
+    g.check_errors()
+
+
+@pytest.mark.parametrize("M,N,K,r", [(256, 512, 512, 32), (300, 528, 768, 16), (129, 400, 320, 64),
+                                     (520, 1296, 1536, 128)])
+def test_unfused_pipeline_matches_oracle(M, N, K, r):
+    # In-house unfused form of the layer: quantize without the branch, a separate down-projection that
+    # re-reads X, the plain NVFP4 GEMM, a separate up-projection that reads and rewrites Y.  In fp32
+    # output the literal gate applies.
+    from w4a4_rank_absorbed_b200 import svdq as C
+    wl = small_case(M, K, N, r, seed=19 + M + N + r)
+    dec = oracle_layer(wl, r)
+    g = GpuLayer(dec, wl.bias)
+    X = bf16_dev(wl.X)
+    Xq = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    SFx = torch.empty(C.svdq_sf_bytes(M, K), dtype=torch.uint8, device="cuda")
+    C.svdq_quantize_act(X, M, K, g.inv_s, float(g.gs_x), None, 0, 1.0, Xq, SFx, None)
+    LA = torch.empty((M, 2 * r), dtype=torch.bfloat16, device="cuda")
+    C.svdq_lowrank_down(X, M, K, g.L1fT, r, 1.0, LA, C.new_workspace(M, K, r))
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    C.svdq_linear(Xq, SFx, float(g.gs_x), g.Wq, g.SFw, float(g.gs_w), None, None, 0, g.bias, Y, 1, M, N, K)
+    C.svdq_lowrank_up(LA, g.L2p, r, 1.0, Y, 1, M, N)
+    torch.cuda.synchronize()
+    g.check_errors()
+    Y_or, qa, _ = OL.svdq_reference(wl.X, dec.inv_s, dec.gs_x, dec.L1f, dec.L2b, dec.R32, wl.bias)
+    _assert_bytes(Xq, oracle_storage(qa=qa)["Xq"], "Xq")
+    check_y(Y.cpu().numpy().astype(np.float64), Y_or, bf16=False, what=f"unfused {M}x{N}x{K} r={r}")
+
+
+def test_workspace_is_reusable_and_left_clean():
+    # The ticket words of the workspace return to 0 after every call, so one zeroed workspace serves
+    # any number of calls (and shapes no larger than it was sized for); results repeat bit for bit.
+    from w4a4_rank_absorbed_b200 import svdq as C
+    M, K, r = 640, 2048, 32
+    wl = small_case(M, K, 64, r, seed=99)
+    dec = oracle_layer(wl, r)
+    g = GpuLayer(dec, wl.bias)
+    ws = C.new_workspace(M, K, r)
+    X = bf16_dev(wl.X)
+    outs = []
+    for _ in range(3):
+        Xq = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        SFx = torch.empty(C.svdq_sf_bytes(M, K), dtype=torch.uint8, device="cuda")
+        LAs = torch.empty((M, 2 * r), dtype=torch.bfloat16, device="cuda")
+        C.svdq_quantize_act(X, M, K, g.inv_s, float(g.gs_x), g.L1fT, r, float(g.lr_scale), Xq, SFx, LAs, ws)
+        torch.cuda.synchronize()
+        outs.append((Xq.cpu(), SFx.cpu(), LAs.view(torch.int16).cpu()))
+        tickets = ws[:256].cpu()
+        assert int(tickets.sum()) == 0
+    for o in outs[1:]:
+        assert all(torch.equal(a, b) for a, b in zip(o, outs[0]))
+    check_las(outs[0][2].view(torch.bfloat16), wl.X, dec.L1f, g.lr_scale)
     g.check_errors()

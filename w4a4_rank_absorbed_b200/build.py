@@ -20,7 +20,7 @@ ROOT = os.path.dirname(PKG_DIR)
 SRC = os.path.join(PKG_DIR, "csrc", "svdq.cu")
 OUT = os.path.join(PKG_DIR, "libsvdq.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-# k_linear and k_linear_pair move registers between their warpgroups with setmaxnreg; the split adds up to
+# k_linear moves registers between their warpgroups with setmaxnreg; the split adds up to
 # 512 threads x 128 registers, so the kernel must be launched with exactly 128 a thread
 # (fewer at launch and a warpgroup's setmaxnreg.inc would wait for registers forever).
 LINEAR_ENTRY_REGS = 128
@@ -56,7 +56,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stdout.write(res.stdout + res.stderr)
-    for kernel in ("8k_linearE", "13k_linear_pairE"):
+    for kernel in ("8k_linearE",):
         regs = entry_registers(res.stdout + res.stderr, kernel)
         if regs != LINEAR_ENTRY_REGS:
             os.remove(OUT + ".tmp")

@@ -276,6 +276,26 @@ SVDQ_DEV void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
 }
+// Each thread of the warp reads 16 consecutive 32-bit columns of its TMEM lane.
+SVDQ_DEV void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+SVDQ_DEV void reg_fence16(uint32_t (&v)[16]) {
+  asm volatile(""
+      : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+        "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]));
+}
+// 16-byte store into the shared memory of the cluster CTA whose shared::cluster address is `addr`.
+SVDQ_DEV void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
 // Each thread of the warp writes 16 consecutive 32-bit columns of its TMEM lane.
 SVDQ_DEV void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
@@ -324,6 +344,24 @@ SVDQ_DEV uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Same for a K-major tile whose rows are 64 bytes, stored with the 64-byte swizzle (8-row groups
+// 512 bytes apart, tile base 512-aligned).
+SVDQ_DEV uint64_t sdesc_kmajor_sw64(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(512u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)4u << 61;            // 64-byte swizzle
+  return d;
+}
+
+// ------------------------------------------------- programmatic dependent launch ---
+// Wait until the kernels this grid depends on (launched before it on the stream) have finished and
+// their writes are visible; a no-op when the grid was launched without the programmatic attribute.
+SVDQ_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream start its prologue while this grid runs (it still waits for
+// this grid's completion before reading anything).
+SVDQ_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Instruction descriptor, kind::mxf4nvf4: A, B = E2M1 (K-major), scales UE4M3, M x N, dense K = 64.
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {

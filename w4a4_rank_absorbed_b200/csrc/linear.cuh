@@ -9,7 +9,11 @@
 //   acc  = sum over K tiles of  tcgen05.mma.kind::mxf4nvf4 (A = Xq, B = Wq, scales SFx, SFw)
 //        + sum over rank tiles of tcgen05.mma.kind::f16 (A = LAs, B = L2p)        (same TMEM accumulator)
 //   Y    = f32(gs_x gs_w) * acc + bias
-// LAs was pre-scaled by 1/(gs_x gs_w) in kernel 2, so a single scale serves both branches.
+// LAs was pre-scaled by 1/(gs_x gs_w) in kernel 2, so a single scale serves both branches.  It holds
+// a bf16 hi/lo pair of every low-rank value, interleaved by 16 columns (hi of columns 16j..16j+15,
+// then their lo), so a 64-column LAs box meets one 32-column box of L2p (N x r, a single copy of
+// L2, 64-byte swizzle) twice: MMA k-steps 0 and 1 (hi, lo of columns 0-15 of the box) both read
+// L2p columns 0-15, k-steps 2 and 3 columns 16-31.
 //
 // Persistent, warp-specialised kernel, one CTA of 16 warps per SM, 128 x 256 output tiles:
 //   warp 0   TMA producer for A (box 128 rows x 128 B, 128-byte swizzle) and B (two boxes
@@ -41,6 +45,8 @@ constexpr int LN_STAGES = 4;
 constexpr int LN_A_BYTES = LN_BM * 128;          // 128 rows x 256 FP4 (or 64 bf16)
 constexpr int LN_B_BYTES = LN_BN * 128;
 constexpr int LN_B_HALF = LN_B_BYTES / 2;
+constexpr int LN_LR_B_HALF = 128 * 64;           // rank stage: 128 rows of L2p x 32 bf16 (64-byte rows)
+constexpr int LN_LR_BYTES = LN_A_BYTES + 2 * LN_LR_B_HALF;
 constexpr int LN_SFA_BYTES = 4 * 512;            // 4 K-atoms of 128 rows
 constexpr int LN_SFB_BYTES = 2 * 4 * 512;        // 2 row blocks x 4 K-atoms
 constexpr int LN_THREADS = 512;
@@ -63,8 +69,8 @@ static_assert(LN_SF_COL0 + LN_STAGES * LN_SF_COLS_PER_STAGE <= LN_TMEM_COLS, "TM
 static_assert(LN_STAGES * LN_STREAMS <= 32 && LN_STREAMS == 3, "one lane per slot and stream");
 static_assert(LN_REGS_LOW * 256 + LN_REGS_HIGH * 256 == LN_THREADS * 128, "register split = launch budget");
 
-// Test hooks (svdq_linear_debug): no loads (a forced time-out), force one kernel or the other.
-enum : int { LN_DBG_NO_LOADS = 1, LN_DBG_FORCE_SINGLE = 2, LN_DBG_FORCE_PAIR = 4 };
+// Test hook (svdq_linear_debug): the load warp issues nothing, so the first wait must run out.
+enum : int { LN_DBG_NO_LOADS = 1 };
 
 #ifndef LN_RASTER_GM
 #define LN_RASTER_GM 12
@@ -87,6 +93,7 @@ struct LinearArgs {
   void* Y;
   int y_fp32;
   int y_vec32;          // Y is 32-byte aligned: 32-byte stores
+  int y_accum;          // Y += result (read-modify-write, the unfused up-projection); no bias
 
   int M, N, K, r;
   float gs;
@@ -106,7 +113,28 @@ SVDQ_DEV void store_y_row(const LinearArgs& a, const uint32_t (&v)[4][32], int r
       const int n = n0 + 32 * i + 16 * gp;
       if (n < a.N) {
         float y[16];
-        if (a.bias) {
+        if (a.y_accum) {
+          if (a.y_fp32) {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.Y) + (int64_t)row * a.N + n);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float4 o = src[e];
+              y[4 * e] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 4 * e]), o.x);
+              y[4 * e + 1] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 4 * e + 1]), o.y);
+              y[4 * e + 2] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 4 * e + 2]), o.z);
+              y[4 * e + 3] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 4 * e + 3]), o.w);
+            }
+          } else {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.Y) + (int64_t)row * a.N + n);
+            const uint4 o0 = src[0], o1 = src[1];
+            const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              y[2 * e] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 2 * e]), bf16_lo(ow[e]));
+              y[2 * e + 1] = __fmaf_rn(gs, __uint_as_float(v[i][16 * gp + 2 * e + 1]), bf16_hi(ow[e]));
+            }
+          }
+        } else if (a.bias) {
           const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
           const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 8));
           const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
@@ -155,7 +183,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     const __grid_constant__ CUtensorMap tm_xq,   // uint8 {K/2, M},  box {128, 128}, SW128
     const __grid_constant__ CUtensorMap tm_wq,   // uint8 {K/2, N},  box {128, 128}, SW128
     const __grid_constant__ CUtensorMap tm_las,  // bf16  {2r, M},   box {64, 128},  SW128
-    const __grid_constant__ CUtensorMap tm_l2p,  // bf16  {2r, N},   box {64, 128},  SW128
+    const __grid_constant__ CUtensorMap tm_l2p,  // bf16  {r, N},    box {32, 128},  SW64
     const LinearArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -208,6 +236,10 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  // Everything above overlaps the previous kernel on the stream when launched as a programmatic
+  // dependent; every read of the inputs and every write of Y comes after this wait.
+  griddep_wait();
+  griddep_launch_dependents();
 
   // Register split by warpgroup: every warp of a warpgroup executes the same setmaxnreg, at
   // the top of its role so that the role's code is compiled under that budget.
@@ -255,10 +287,12 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
           const bool lr = kt >= nkt;               // a rank stage: LAs x L2p in bf16
           if (tensor_warp) {
             if (mine) {
-              if (k == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(LN_A_BYTES + LN_B_BYTES));
+              if (k == 0)
+                mbar_arrive_expect_tx(&full[stage], (uint32_t)(lr ? LN_LR_BYTES : LN_A_BYTES + LN_B_BYTES));
               const CUtensorMap* map = k == 0 ? (lr ? &tm_las : &tm_xq) : (lr ? &tm_l2p : &tm_wq);
-              uint8_t* dst = k == 0 ? sA + stage * LN_A_BYTES : sB + stage * LN_B_BYTES + (k - 1) * LN_B_HALF;
-              const int x = lr ? (kt - nkt) * 64 : kt * 128;
+              uint8_t* dst = k == 0 ? sA + stage * LN_A_BYTES
+                                    : sB + stage * LN_B_BYTES + (k - 1) * (lr ? LN_LR_B_HALF : LN_B_HALF);
+              const int x = lr ? (kt - nkt) * (k == 0 ? 64 : 32) : kt * 128;
               const int y = k == 0 ? mb * LN_BM : nb * LN_BN + (k - 1) * 128;
               __syncwarp(smask);
               tma_load_2d(dst, map, &full[stage], x, y);
@@ -325,8 +359,12 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
               tc_mma_nvf4(tbase, adesc + 2 * j, bdesc + 2 * j, IDESC_F4, sfa_col + 4 * j, sfb_col + 8 * j,
                           (kt | j) != 0 ? 1u : 0u);
           } else {
+            // hi and lo of the same 16 low-rank columns meet the same 16 columns of L2p.  (With no
+            // K tiles, the rank-only mode, the first rank MMA starts the accumulator.)
+            const uint64_t bdesc64 = sdesc_kmajor_sw64(smem_u32(sB + stage * LN_B_BYTES));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tc_mma_bf16(tbase, adesc + 2 * j, bdesc + 2 * j, IDESC_BF16, 1u);
+            for (int j = 0; j < 4; ++j)
+              tc_mma_bf16(tbase, adesc + 2 * j, bdesc64 + 2 * (j >> 1), IDESC_BF16, (kt | j) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           if (++stage == LN_STAGES) { stage = 0; phase ^= 1u; }

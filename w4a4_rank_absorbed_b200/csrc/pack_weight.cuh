@@ -11,8 +11,8 @@
 //   2. amax |R| over the whole tensor (vectorised grid-stride loads, atomicMax on the bits);
 //   3. gs_w = amax / 2688 (or 1);
 //   4. encode: one thread per (column n, 64 consecutive k): 4 groups of 16,
-//      32 bytes of codes and one 32-bit word of scales; also the doubled
-//      up-projection layout L2p (N x 2r).
+//      32 bytes of codes and one 32-bit word of scales; also the up-projection
+//      laid out K-major for the GEMM, L2p = L2^T (N x r).
 #pragma once
 #include "common.cuh"
 
@@ -109,16 +109,45 @@ __global__ void __launch_bounds__(128) k_pack_weight(const float* __restrict__ R
   *reinterpret_cast<uint32_t*>(sfw) = sfword;
 }
 
-// L2p[n, j] = L2b[j mod r, n] for j < 2r.  grid: ceil(N/128); block 128.
+// Q(R) from a packed weight: R_q[k, n] = f32(e2m1(code) * f32(dec(sb) * gs)), K x N row-major.
+// grid: (ceil(N/128), K/64); block 128; thread = (column n, 64-row slab kb), so a warp writes 32
+// consecutive columns of one row at a time.
+__global__ void __launch_bounds__(128) k_dequant_weight(const uint8_t* __restrict__ Wq,
+                                                        const uint8_t* __restrict__ SFw,
+                                                        const float* __restrict__ gs_ptr, int K, int N,
+                                                        float* __restrict__ Rq) {
+  const int n = blockIdx.x * 128 + threadIdx.x;
+  const int kb = blockIdx.y;
+  if (n >= N) return;
+  const float gs = *gs_ptr;
+  const uint32_t sfword = *reinterpret_cast<const uint32_t*>(SFw + sf_word_offset((uint32_t)n, (uint32_t)kb,
+                                                                                  (uint32_t)(K >> 6)));
+  const uint4* src = reinterpret_cast<const uint4*>(Wq + (int64_t)n * (K >> 1) + kb * 32);
+  const uint4 c0 = src[0], c1 = src[1];
+  const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  // E2M1 magnitudes of codes 0..7 (bit 3 is the sign)
+  const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const float d = __fmul_rn(dec_ue4m3((sfword >> (8 * g)) & 0xFFu), gs);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t code = (cw[2 * g + (i >> 3)] >> (4 * (i & 7))) & 0xFu;
+      const float v = __fmul_rn(mag[code & 7u], d);
+      Rq[(int64_t)(kb * 64 + g * 16 + i) * N + n] = (code & 8u) ? -v : v;
+    }
+  }
+}
+
+// L2p[n, t] = L2b[t, n] for t < r (r even).  grid: ceil(N/128); block 128.
 __global__ void __launch_bounds__(128) k_layout_l2(const uint16_t* __restrict__ L2b, int N, int r,
                                                    uint16_t* __restrict__ L2p) {
   const int n = blockIdx.x * 128 + threadIdx.x;
   if (n >= N) return;
-  uint16_t* row = L2p + (int64_t)n * 2 * r;
+  uint16_t* row = L2p + (int64_t)n * r;
   for (int t = 0; t < r; t += 2) {
     const uint32_t v = (uint32_t)L2b[(int64_t)t * N + n] | ((uint32_t)L2b[(int64_t)(t + 1) * N + n] << 16);
     *reinterpret_cast<uint32_t*>(row + t) = v;
-    *reinterpret_cast<uint32_t*>(row + r + t) = v;
   }
 }
 

@@ -3,86 +3,73 @@
 // SVDQuant review, §4.3 (Nunchaku): the down-projection is merged into the
 // quantization kernel, so the 16-bit activations are read from HBM once and
 // shared by both branches.  Per element x_hat = f32(x * inv_s) (the smoothing
-// divide, "From SmoothQuant to SVDQuant", section Smooth Quant (W8A8));
-// per group of 16 along K the NVFP4 codec of SVDQuant review §3 (q_max = 6)
-// with a UE4M3 block scale; the down-projection LA = X L1f (L1f =
-// diag(s)^-1 L1, so X L1f = X_hat L1) on the tensor cores (bf16 in, fp32
-// accumulate), pre-scaled by lr_scale and split into bf16 hi/lo halves.
+// divide, "From SmoothQuant to SVDQuant", section Smooth Quant (W8A8)); per
+// group of 16 along K the NVFP4 codec of SVDQuant review §3 (q_max = 6) with a
+// UE4M3 block scale; the down-projection LA = X L1f (L1f = diag(s)^-1 L1, so
+// X L1f = X_hat L1) on the tcgen05 tensor cores (bf16 in, fp32 accumulate in
+// TMEM), pre-scaled by lr_scale and split into bf16 hi/lo halves.
 //
-// CTA = 32 rows x all of K; 14 warps in 7 pairs.  The K axis is cut into
-// 64-column chunks; chunk c goes through ring stage c % S and is consumed by
-// warp pair c % 7, so seven chunks are processed at once.  S is a multiple of
-// 7 (up to 49): as many stages as fit in 200 KB, 21 for r = 32, 7 for r = 128,
-// so each pair keeps S/7 chunks in flight.  A pair loads its own chunks: once
-// both of its warps are done with a stage, warp 0 of the pair issues the copies
-// of the chunk S further on into that stage (three lanes in one converged
-// instruction, rotating with the round so no thread has two copies in flight:
-// a thread's copies are serviced one after another).  No producer warp, and no
-// lanes waiting on different barriers in divergent branches.  A stage holds
-// the X box (32 x 64 bf16, 128-byte swizzle), the L1f^T box (r x 64 bf16, same
-// swizzle) and the chunk's 64 smoothing factors.  Warp h of a pair owns rows
-// 16h..16h+15 of the chunk: two lanes per row quantize two groups of 16 each,
-// and the warp runs the 16 x r down-projection of its rows for the chunk's 64
-// columns (mma.sync m16n8k16), keeping a partial sum in registers.  After the
-// last chunk the seven partial sums of every row are added in shared memory and
-// written as LAs.
+// Work split: a CTA owns 128 rows and a contiguous range of the K axis; `split`
+// CTAs share a row block (split = 1 when there are enough row blocks to fill
+// the GPU).  The K axis is read in 64-column chunks through an S-stage ring
+// (TMA, 128-byte swizzle): the 128 x 64 X box, the r x 64 L1f^T box and the
+// chunk's 64 smoothing factors.  Roles (18 warps):
+//   warp 0      producer: three lanes issue a stage's three copies in one
+//               converged instruction; the lanes rotate with the ring slot so no
+//               thread has two copies of one stream in flight.
+//   warp 1      TMEM owner and MMA issuer (one thread): per chunk four
+//               tcgen05.mma.kind::f16 of 128 x r x 16 (A = the X box, B = the
+//               L1f^T box) into one fp32 accumulator of r TMEM columns; each
+//               chunk's commit is one of the arrivals that frees its stage.
+//   warps 2-17  quantizers: thread i takes row i / 4, group i % 4 of the chunk
+//               (16 values), writes 8 bytes of codes and, gathered over the
+//               row's four lanes, one 32-bit word of scales.
+// After the last chunk, four of the quantizer warps (one per TMEM lane quarter)
+// read the accumulator.  With split = 1 it goes through shared memory straight
+// to LAs.  Otherwise each CTA writes its partial sums to the caller's workspace
+// and takes a ticket for its row block; the CTA that takes the last ticket adds
+// the `split` partials in rank order (the result does not depend on which CTA
+// finishes last) and resets the ticket to 0 for the next call.  LAs holds the
+// hi/lo pair of lr_scale * (X L1f), interleaved by 16 columns (hi of columns
+// 16j..16j+15 at 32j, their lo at 32j + 16), the order the GEMM's rank stage
+// reads.
+//
+// With QUANT = false the same kernel is the separate down-projection of the
+// unfused pipeline (the quantizer warps only release the stages).
 #pragma once
 #include "common.cuh"
 
 namespace svdq {
 
-constexpr int QA_ROWS = 32;
-constexpr int QA_CHUNK = 64;          // bf16 columns per chunk (128 bytes)
-constexpr int QA_PAIRS = 7;
-constexpr int QA_CONSUMER_WARPS = 2 * QA_PAIRS;
-constexpr int QA_THREADS = QA_CONSUMER_WARPS * 32;
-constexpr int QA_RING_BYTES = 200 * 1024;
+constexpr int QB_ROWS = 128;
+constexpr int QB_CHUNK = 64;                 // bf16 columns per chunk (128 bytes)
+constexpr int QB_QWARPS = 16;
+constexpr int QB_WARP_Q0 = 2;                // first quantizer warp
+constexpr int QB_THREADS = (QB_WARP_Q0 + QB_QWARPS) * 32;
+constexpr int QB_MAX_SPLIT = 8;                // power of two: 128 rows / split, ticket arithmetic
+constexpr int QB_RING_BYTES = 200 * 1024;
+constexpr int QB_MAX_STAGES = 12;
 
 template <int R>
-struct QaCfg {
-  static constexpr int kXBytes = QA_ROWS * 128;
+struct QbCfg {
+  static constexpr int kXBytes = QB_ROWS * 128;
   static constexpr int kLBytes = R * 128;
-  static constexpr int kStageBytes = kXBytes + kLBytes;
-  // The ring size is a multiple of the pair count, so a ring slot is always loaded and consumed
-  // by the same warp pair, one round after another.
-  static constexpr int kPerPair = QA_RING_BYTES / (QA_PAIRS * (kStageBytes + 256));
-  static constexpr int kStages = QA_PAIRS * (kPerPair < 1 ? 1 : kPerPair > 7 ? 7 : kPerPair);
-  static constexpr int kNT = R / 8;                                  // n8 tiles of the r columns
-  static constexpr int kAcc = R > 0 ? kNT : 1;                      // (m16, n8) tiles per warp
-  static constexpr int kRedBytes = QA_PAIRS * QA_ROWS * R * 4;
+  static constexpr int kInvBytes = 1024;     // 64 floats used; keeps the next stage 1024-aligned
+  static constexpr int kStageBytes = kXBytes + kLBytes + kInvBytes;
+  static constexpr int kStages = QB_RING_BYTES / kStageBytes < QB_MAX_STAGES ? QB_RING_BYTES / kStageBytes
+                                                                             : QB_MAX_STAGES;
   static constexpr int kRingBytes = kStages * kStageBytes;
-  static_assert(kRedBytes <= kRingBytes, "reduction buffer must fit in the ring");
-  static constexpr int kInvOff = kRingBytes;                        // S x 64 smoothing factors
-  static constexpr int kRcpOff = kInvOff + kStages * 256;           // 128-entry 1/d table
+  static_assert(QB_ROWS * R * 4 <= kRingBytes, "the reduction buffer reuses the ring");
+  static_assert(QB_ROWS * R * 4 + 16 <= kRingBytes, "the last-CTA flag sits after it");
+  static constexpr int kRcpOff = kRingBytes;                // 128-entry 1/d table
   static constexpr int kBarOff = kRcpOff + 128 * 4;
-  static constexpr int kSmem = kBarOff + 2 * kStages * 8 + 16 + 1024;
+  static constexpr int kSmem = kBarOff + (2 * kStages + 2) * 8 + 16 + 1024;
+  static constexpr int kTmemCols = R <= 32 ? 32 : R <= 64 ? 64 : 128;
 };
-
-SVDQ_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-SVDQ_DEV void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
-}
-SVDQ_DEV void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                             uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-SVDQ_DEV void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
 
 // Byte offset of 16-byte chunk `c16` of row `row` in a 128-byte-swizzled tile.
 SVDQ_DEV uint32_t sw128(uint32_t row, uint32_t c16) { return row * 128u + ((c16 ^ (row & 7u)) << 4); }
 
-// One group of 16 values of X (two 16-byte smem chunks) times 16 smoothing factors:
-// returns the UE4M3 scale and the two 32-bit code words.
 // d = a * b element-wise on two float32 pairs (two correctly rounded products).
 SVDQ_DEV float2 mul_f32x2(float2 a, float2 b) {
   uint64_t d;
@@ -124,34 +111,51 @@ SVDQ_DEV uint32_t quant_group(const uint4& r0, const uint4& r1, const float4 (&i
   return sb;
 }
 
-template <int R>
-__global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
-    const __grid_constant__ CUtensorMap tm_x,   // bf16 {K, M}, box {64, 32}, 128B swizzle
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
+SVDQ_DEV bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, volatile int* abort, unsigned site) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, timeout_ns, abort, site) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+template <int R, bool QUANT>
+__global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
+    const __grid_constant__ CUtensorMap tm_x,   // bf16 {K, M}, box {64, 128}, 128B swizzle
     const __grid_constant__ CUtensorMap tm_l1,  // bf16 {K, R}, box {64, R}, 128B swizzle
-    const float* __restrict__ inv_s, float gs_x, float lr_scale, int M, int K, int Mpad,
-    uint8_t* __restrict__ Xq, uint8_t* __restrict__ SFx, uint16_t* __restrict__ LAs, uint64_t timeout_ns) {
-  using Cfg = QaCfg<R>;
+    const float* __restrict__ inv_s, float gs_x, float lr_scale, int M, int K, int Mpad, int split,
+    uint8_t* __restrict__ Xq, uint8_t* __restrict__ SFx, uint16_t* __restrict__ LAs,
+    float* __restrict__ ws_part,            // split > 1: [split][Mpad][R] partial sums
+    unsigned int* __restrict__ ws_ticket,   // split > 1: one counter per row block, 0 between calls
+    uint64_t timeout_ns) {
+  using Cfg = QbCfg<R>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* s_inv = reinterpret_cast<float*>(smem + Cfg::kInvOff);
   float* s_rcp = reinterpret_cast<float*>(smem + Cfg::kRcpOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
-  uint64_t* consumed = full + S;           // both warps of the owning pair are done with the stage
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(consumed + S);
+  uint64_t* empty = full + S;              // quantizer warps done and (r > 0) the chunk's MMAs complete
+  uint64_t* acc_full = empty + S;          // every MMA of this CTA complete
+  uint64_t* drain = acc_full + 1;          // MMA thread, on a time-out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * QA_ROWS;
-  const int nchunks = K / QA_CHUNK;
-  const int pairi = warp >> 1;             // warp pair: consumes chunks pairi, pairi + 7, ...
-  const int half = warp & 1;               // rows 16*half .. 16*half + 15 of the chunk
+  const int rank = (int)(blockIdx.x % (unsigned)split);   // position of this CTA in its row block
+  const int rb = (int)(blockIdx.x / (unsigned)split);
+  const int m0 = rb * QB_ROWS;
+  const int nch = K / QB_CHUNK;
+  const int c_begin = rank * nch / split;
+  const int my = (rank + 1) * nch / split - c_begin;       // chunks of this CTA (>= 1)
+  const uint64_t tmo = timeout_ns;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&consumed[s], 2);
+      mbar_init(&empty[s], QB_QWARPS + (R > 0 ? 1 : 0));
     }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -160,148 +164,180 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
     const uint32_t sb = threadIdx.x;
     s_rcp[sb] = sb == 0 ? 0.0f : __frcp_rn(__fmul_rn(dec_ue4m3(sb), gs_x));
   }
+  if constexpr (R > 0) {
+    if (warp == 1) {
+      tmem_alloc(tmem_slot, Cfg::kTmemCols);
+      tmem_relinquish();
+    }
+  }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
     if (R > 0) tma_prefetch_desc(&tm_l1);
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = R > 0 ? *tmem_slot : 0u;
+  // X may be the previous kernel's output: read nothing before it has finished.
+  griddep_wait();
+  griddep_launch_dependents();
 
-  // Copies of chunk c into its stage, by lanes 3j .. 3j + 2 of warp 0 of the owning pair (j
-  // rotates with the round): X box and L1f^T box in one converged instruction, then the chunk's
-  // 64 smoothing factors.
-  auto issue = [&](int c) {
-    const int g = c % S;
-    const int j = (c / S) % 10;
-    if (lane >= 3 * j && lane < 3 * j + 3) {
-      const int k = lane - 3 * j;
-      uint8_t* st = smem + g * Cfg::kStageBytes;
-      if (k == 0) mbar_arrive_expect_tx(&full[g], Cfg::kStageBytes + 256);
-      __syncwarp(7u << (3 * j));
-      if (k == 0 || (k == 1 && R > 0))
-        tma_load_2d(k == 0 ? st : st + Cfg::kXBytes, k == 0 ? &tm_x : &tm_l1, &full[g], c * QA_CHUNK,
-                    k == 0 ? m0 : 0);
-      else if (k == 2)
-        bulk_load(s_inv + g * 64, inv_s + (int64_t)c * QA_CHUNK, 256, &full[g]);
-    }
-    __syncwarp();
-  };
-  int hi = pairi;                          // the pair's chunks below hi have been issued
-  for (; hi < nchunks && hi < S; hi += QA_PAIRS)
-    if (half == 0) issue(hi);
-
-  const int qrow = 16 * half + (lane >> 1);
-  const int qg = 2 * (lane & 1);           // first of the two groups this lane quantizes
-  const int m = m0 + qrow;
-  const float c_x = __frcp_rn(__fmul_rn(6.0f, gs_x));
-  const uint32_t KS4 = (uint32_t)(K >> 6);
-  const uint32_t rcp_u32 = smem_u32(s_rcp);
-
-  float acc[Cfg::kAcc][4];
-#pragma unroll
-  for (int i = 0; i < Cfg::kAcc; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
-
-  bool ok = true;
-  int c = pairi;
-  for (; c < nchunks; c += QA_PAIRS) {
-    const int s = c % S;
-    if (!mbar_wait(&full[s], (uint32_t)((c / S) & 1), timeout_ns, abort_flag, 0x202)) {
-      ok = false;
-      break;
-    }
-    const uint8_t* st = smem + s * Cfg::kStageBytes;
-    const uint32_t st_u32 = smem_u32(st);
-    const uint32_t inv_u32 = smem_u32(s_inv + s * 64 + 16 * qg);
-
-    // ---- quantize two groups of row qrow ------------------------------------
-    uint32_t w[4];
-    uint32_t sb2 = 0u;
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      const int gg = qg + g;
-      const uint4 r0 = lds_v4(st_u32 + sw128(qrow, 2 * gg));
-      const uint4 r1 = lds_v4(st_u32 + sw128(qrow, 2 * gg + 1));
-      float4 inv[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) inv[j] = lds_v4f(inv_u32 + 64 * g + 16 * j);
-      const uint32_t sb = quant_group(r0, r1, inv, c_x, rcp_u32, w[2 * g], w[2 * g + 1]);
-      sb2 |= sb << (8 * g);
-    }
-    const uint32_t other = __shfl_xor_sync(0xffffffffu, sb2, 1);
-    if (m < M)
-      *reinterpret_cast<uint4*>(Xq + (int64_t)m * (K >> 1) + c * 32 + 8 * qg) = make_uint4(w[0], w[1], w[2], w[3]);
-    if ((lane & 1) == 0 && m < Mpad)
-      *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)m, (uint32_t)c, KS4)) = sb2 | (other << 16);
-
-    // ---- down-projection of this warp's 16 rows on the tensor cores ---------
-    if constexpr (R > 0) {
-      const uint32_t sl_u32 = st_u32 + Cfg::kXBytes;
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t a0, a1, a2, a3;
-        const uint32_t arow = 16 * half + (lane & 7) + ((lane >> 3) & 1) * 8;
-        ldsm_x4(st_u32 + sw128(arow, ks * 2 + (lane >> 4)), a0, a1, a2, a3);
-#pragma unroll
-        for (int nt = 0; nt < Cfg::kNT; nt += 2) {
-          uint32_t b[4];
-          const uint32_t brow = (nt + (lane >> 4)) * 8 + (lane & 7);
-          ldsm_x4(sl_u32 + sw128(brow, ks * 2 + ((lane >> 3) & 1)), b[0], b[1], b[2], b[3]);
-          mma_bf16_16816(acc[nt], a0, a1, a2, a3, b[0], b[1]);
-          mma_bf16_16816(acc[nt + 1], a0, a1, a2, a3, b[2], b[3]);
-        }
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer --
+    const int k = lane % 3;
+    int issued = 0;
+    bool ok = true;
+    for (int i = 0; i < my; ++i) {
+      const int s = i % S;
+      if (i >= S && !warp_wait(&empty[s], (uint32_t)(((i / S) - 1) & 1), tmo, abort_flag, 0x201)) {
+        ok = false;
+        break;
       }
-    }
-    // Once both warps of the pair are done with stage s, warp 0 refills it with the chunk S
-    // further on.
-    if (c + S < nchunks) {
+      const int g = s % 10;                   // lanes 3g .. 3g + 2 serve slot s
+      if (lane >= 3 * g && lane < 3 * g + 3) {
+        uint8_t* st = smem + s * Cfg::kStageBytes;
+        const int c = c_begin + i;
+        if (k == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(Cfg::kXBytes + Cfg::kLBytes + (QUANT ? 256 : 0)));
+        __syncwarp(7u << (3 * g));
+        if (k == 0)
+          tma_load_2d(st, &tm_x, &full[s], c * QB_CHUNK, m0);
+        else if (k == 1 && R > 0)
+          tma_load_2d(st + Cfg::kXBytes, &tm_l1, &full[s], c * QB_CHUNK, 0);
+        else if (k == 2 && QUANT)
+          bulk_load(st + Cfg::kXBytes + Cfg::kLBytes, inv_s + (int64_t)c * QB_CHUNK, 256, &full[s]);
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&consumed[s]);
-      if (half == 0) {
-        int done = 1;
-        if (lane == 0) done = mbar_wait(&consumed[s], (uint32_t)((c / S) & 1), timeout_ns, abort_flag, 0x201) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, done, 0)) {
-          ok = false;
-          c += QA_PAIRS;                   // chunk c was consumed; the loads still owed start after it
-          break;
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue(c + S);
-      }
-      hi = c + S + QA_PAIRS;
+      issued = i + 1;
     }
-  }
-  if (!ok && half == 0) {
-    // Let the loads this pair issued but did not consume land before the CTA exits.
-    int never = 0;
-    for (int c2 = c; c2 < hi; c2 += QA_PAIRS)
-      mbar_wait(&full[c2 % S], (uint32_t)((c2 / S) & 1), timeout_ns, &never, 0x203);
+    if (!ok && lane == 0) {
+      // Let the copies that were issued but not consumed land before the CTA exits.
+      int never = 0;
+      for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+        mbar_wait(&full[i % S], (uint32_t)((i / S) & 1), tmo, &never, 0x203);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer --
+    if constexpr (R > 0) {
+      if (lane == 0) {
+        constexpr uint32_t IDESC = idesc_bf16(QB_ROWS, R);
+        bool ok = true;
+        for (int i = 0; i < my; ++i) {
+          const int s = i % S;
+          if (!mbar_wait(&full[s], (uint32_t)((i / S) & 1), tmo, abort_flag, 0x211)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* st = smem + s * Cfg::kStageBytes;
+          const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(st));
+          const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(st + Cfg::kXBytes));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tc_mma_bf16(tbase, adesc + 2 * j, bdesc + 2 * j, IDESC, (i | j) != 0 ? 1u : 0u);
+          tc_commit(&empty[s]);
+        }
+        if (ok) {
+          tc_commit(acc_full);
+          // The ring becomes the reduction buffer: the MMAs must have finished reading it.
+          ok = mbar_wait(acc_full, 0, tmo, abort_flag, 0x212);
+        }
+        if (!ok || *abort_flag) {
+          int never = 0;
+          tc_commit(drain);
+          mbar_wait(drain, 0, tmo, &never, 0x213);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ quantizers --
+    const int qi = threadIdx.x - QB_WARP_Q0 * 32;
+    const int row = qi >> 2;
+    const int g = qi & 3;
+    const int m = m0 + row;
+    const float c_x = __frcp_rn(__fmul_rn(6.0f, gs_x));
+    const uint32_t KS4 = (uint32_t)(K >> 6);
+    const uint32_t rcp_u32 = smem_u32(s_rcp);
+    for (int i = 0; i < my; ++i) {
+      const int s = i % S;
+      if (!warp_wait(&full[s], (uint32_t)((i / S) & 1), tmo, abort_flag, 0x202)) break;
+      if constexpr (QUANT) {
+        const int c = c_begin + i;
+        const uint32_t st_u32 = smem_u32(smem + s * Cfg::kStageBytes);
+        const uint32_t inv_u32 = st_u32 + Cfg::kXBytes + Cfg::kLBytes + 64 * g;
+        const uint4 r0 = lds_v4(st_u32 + sw128(row, 2 * g));
+        const uint4 r1 = lds_v4(st_u32 + sw128(row, 2 * g + 1));
+        float4 inv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) inv[j] = lds_v4f(inv_u32 + 16 * j);
+        uint32_t w0, w1;
+        uint32_t sw = quant_group(r0, r1, inv, c_x, rcp_u32, w0, w1) << (8 * g);
+        sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
+        sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
+        if (m < M) *reinterpret_cast<uint2*>(Xq + (int64_t)m * (K >> 1) + c * 32 + 8 * g) = make_uint2(w0, w1);
+        if (g == 0 && m < Mpad)
+          *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)m, (uint32_t)c, KS4)) = sw;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
   }
 
-  // ---- LAs = [hi | lo] of lr_scale * sum over pairs of the partial X L1f ----
+  // ---- LAs = hi/lo of lr_scale * (sum over the row block's CTAs of the partial X L1f) ----
   if constexpr (R > 0) {
-    // Every chunk has been consumed, so no load is in flight into the ring: reuse it.
-    named_bar_sync(1, QA_CONSUMER_WARPS * 32);
-    float* red = reinterpret_cast<float*>(smem);            // [pair][row][R]
-    if (ok) {
+    // Every chunk has been consumed and every MMA has finished (or the CTA gave up), so the ring
+    // is idle: with split = 1 it holds the accumulator rows, red[row][R].
+    tc_fence_before();
+    __syncthreads();
+    float* red = reinterpret_cast<float*>(smem);
+    volatile int* s_last = reinterpret_cast<volatile int*>(smem + QB_ROWS * R * 4);
+    if (warp >= QB_WARP_Q0 && warp < QB_WARP_Q0 + 4) {
+      const int q = warp & 3;                // TMEM lane quarter of this warp
+      if (warp_wait(acc_full, 0, tmo, abort_flag, 0x221)) {
+        tc_fence_after();
+        const int row = 32 * q + lane;
+        float* dst = split > 1 ? ws_part + ((size_t)rank * Mpad + m0 + row) * R : red + (size_t)row * R;
 #pragma unroll
-      for (int nt = 0; nt < Cfg::kNT; ++nt) {
-        const int row = 16 * half + (lane >> 2);
-        const int col = nt * 8 + 2 * (lane & 3);
-        float* p = red + ((pairi * QA_ROWS + row) * R + col);
-        *reinterpret_cast<float2*>(p) = make_float2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<float2*>(p + 8 * R) = make_float2(acc[nt][2], acc[nt][3]);
+        for (int cc = 0; cc < R / 16; ++cc) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tbase + ((uint32_t)(32 * q) << 16) + 16 * cc, v);
+          tmem_ld_wait();
+          reg_fence16(v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            reinterpret_cast<uint4*>(dst + 16 * cc)[e] = make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        }
       }
     }
-    named_bar_sync(1, QA_CONSUMER_WARPS * 32);
-    if (ok && !*abort_flag) {
-      for (int p = threadIdx.x; p < QA_ROWS * R / 2; p += QA_CONSUMER_WARPS * 32) {
+    tc_fence_before();
+    if (split > 1) {
+      // Publish this CTA's partial, then take a ticket; the CTA that takes the last one reduces.
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const unsigned old = atomicAdd(&ws_ticket[rb], 1u);
+        const int last = (old % (unsigned)split) == (unsigned)split - 1u;
+        if (last) atomicExch(&ws_ticket[rb], 0u);
+        *s_last = last;
+      }
+      __syncthreads();
+      __threadfence();
+    } else {
+      __syncthreads();
+    }
+    if (!*abort_flag && (split == 1 || *s_last)) {
+      for (int p = threadIdx.x; p < QB_ROWS * (R / 2); p += QB_THREADS) {
         const int row = p / (R / 2);
         const int col = 2 * (p % (R / 2));
         float v0 = 0.0f, v1 = 0.0f;
-#pragma unroll
-        for (int w2 = 0; w2 < QA_PAIRS; ++w2) {
-          const float2 t = *reinterpret_cast<const float2*>(red + ((w2 * QA_ROWS + row) * R + col));
-          v0 += t.x;
-          v1 += t.y;
+        if (split == 1) {
+          const float2 t = *reinterpret_cast<const float2*>(red + (size_t)row * R + col);
+          v0 = t.x;
+          v1 = t.y;
+        } else {
+          for (int src = 0; src < split; ++src) {
+            const float2 t = __ldcg(reinterpret_cast<const float2*>(ws_part + ((size_t)src * Mpad + m0 + row) * R + col));
+            v0 += t.x;
+            v1 += t.y;
+          }
         }
         const int mm = m0 + row;
         if (mm < M) {
@@ -309,11 +345,15 @@ __global__ void __launch_bounds__(QA_THREADS, 1) k_quantize_act(
           v1 = __fmul_rn(v1, lr_scale);
           const float h0 = __bfloat162float(__float2bfloat16_rn(v0));
           const float h1 = __bfloat162float(__float2bfloat16_rn(v1));
-          uint16_t* dst = LAs + (int64_t)mm * (2 * R);
-          *reinterpret_cast<uint32_t*>(dst + col) = pack_bf16x2(h0, h1);
-          *reinterpret_cast<uint32_t*>(dst + R + col) = pack_bf16x2(v0 - h0, v1 - h1);
+          uint16_t* d = LAs + (int64_t)mm * (2 * R) + 32 * (col >> 4) + (col & 15);
+          *reinterpret_cast<uint32_t*>(d) = pack_bf16x2(h0, h1);
+          *reinterpret_cast<uint32_t*>(d + 16) = pack_bf16x2(v0 - h0, v1 - h1);
         }
       }
+    }
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tbase, Cfg::kTmemCols);
     }
   }
 }

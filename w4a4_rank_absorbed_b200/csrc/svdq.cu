@@ -8,11 +8,11 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/svdq.h"
 #include "common.cuh"
 #include "linear.cuh"
-#include "linear_pair.cuh"
 #include "pack_weight.cuh"
 #include "quantize_act.cuh"
 
@@ -28,8 +28,7 @@ struct DevInfo {
   bool ok = false;
   int sms = 0;
   bool linear_attr = false;
-  bool linear_pair_attr = false;
-  bool qa_attr[9] = {};
+  bool qa_attr[2][9] = {};
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -74,9 +73,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor (rows x inner elements, row pitch in bytes), box (box_inner x box_rows), 128B swizzle.
+// 2-D row-major tensor (rows x inner elements, row pitch in bytes), box (box_inner x box_rows),
+// 128-byte swizzle unless stated.
 bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
-                 uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows) {
+                 uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows,
+                 CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
@@ -84,7 +85,7 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -106,14 +107,59 @@ svdq_status launch_status() {
 
 int64_t pad128(int64_t v) { return (v + 127) / 128 * 128; }
 
+// Launch as a programmatic dependent of the previous kernel on the stream: the kernel's prologue
+// (barrier set-up, TMEM allocation, descriptor prefetch) overlaps that kernel's tail, and the kernel
+// waits for it (griddepcontrol.wait) before it touches global memory.  cluster > 1 launches
+// thread-block clusters of that many CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // --------------------------------------------------------- quantize_act -----
-template <int R>
-svdq_status launch_qa(DevInfo* d, int slot, const uint16_t* X, int64_t M, int64_t K, const float* inv_s,
-                      float gs_x, const uint16_t* L1fT, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
-                      cudaStream_t s) {
-  using Cfg = QaCfg<R>;
+// CTAs that share a 128-row block split its K chunks between them: the smallest split in
+// {1, 2, 4, 8} that gives about one CTA per SM (the kernel runs one 576-thread CTA per SM, so a
+// larger grid would run in two waves), with at least two chunks a CTA.
+int qa_split(int64_t M, int64_t K, int sms) {
+  const int64_t rb = pad128(M) / 128, nch = K / 64;
+  int split = 1;
+  while (split < QB_MAX_SPLIT && rb * 2 * split <= (int64_t)sms && nch >= 4 * split) split *= 2;
+  return split;
+}
+
+// Workspace of kernel 2 (see include/svdq.h): the ticket words first, then the partial sums.
+size_t qa_ticket_bytes(int64_t M) { return (size_t)((pad128(M) / 128 * 4 + 255) / 256 * 256); }
+size_t qa_workspace_bytes(int64_t M, int r) {
+  return r > 0 ? qa_ticket_bytes(M) + (size_t)QB_MAX_SPLIT * (size_t)pad128(M) * (size_t)r * 4 : 0;
+}
+
+template <int R, bool QUANT>
+svdq_status launch_qa(DevInfo* d, const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float gs_x,
+                      const uint16_t* L1fT, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
+                      void* ws, cudaStream_t s) {
+  using Cfg = QbCfg<R>;
   CUtensorMap tm_x, tm_l1;
-  if (!make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 32))
+  if (!make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64,
+                   QB_ROWS))
     return SVDQ_ERR_CUDA;
   if (R > 0) {
     if (!make_map_2d(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1fT, (uint64_t)K, (uint64_t)R, (uint64_t)K * 2, 64,
@@ -122,28 +168,58 @@ svdq_status launch_qa(DevInfo* d, int slot, const uint16_t* X, int64_t M, int64_
   } else {
     tm_l1 = tm_x;
   }
-  if (!d->qa_attr[slot]) {
-    if (cudaFuncSetAttribute(k_quantize_act<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
+  bool& attr = d->qa_attr[QUANT ? 0 : 1][R / 16];
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_quantize_act<R, QUANT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
         cudaSuccess)
       return SVDQ_ERR_CUDA;
-    d->qa_attr[slot] = true;
+    attr = true;
   }
   const int64_t Mpad = pad128(M);
-  const dim3 grid((unsigned)(Mpad / QA_ROWS));
-  k_quantize_act<R><<<grid, QA_THREADS, Cfg::kSmem, s>>>(tm_x, tm_l1, inv_s, gs_x, lr_scale, (int)M, (int)K,
-                                                         (int)Mpad, Xq, SFx, LAs, LN_DEFAULT_TIMEOUT_NS);
+  const int split = qa_split(M, K, d->sms);   // with r = 0 the CTAs of a row block only share out K
+  unsigned int* ticket = reinterpret_cast<unsigned int*>(ws);
+  float* part = ws ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + qa_ticket_bytes(M)) : nullptr;
+  if (R > 0 && split > 1 && !ws) return SVDQ_ERR_INVALID_ARG;
+  const dim3 grid((unsigned)(Mpad / QB_ROWS * split));
+  if (launch_pdl(k_quantize_act<R, QUANT>, grid, dim3(QB_THREADS), (size_t)Cfg::kSmem, s, 1, tm_x, tm_l1,
+                 inv_s, gs_x, lr_scale, (int)M, (int)K, (int)Mpad, split, Xq, SFx, LAs, part, ticket,
+                 LN_DEFAULT_TIMEOUT_NS) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
   return launch_status();
+}
+
+template <bool QUANT>
+svdq_status dispatch_qa(DevInfo* d, int r, const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float gs_x,
+                        const uint16_t* L1fT, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
+                        void* ws, cudaStream_t s) {
+  switch (r) {
+    case 0:
+      if (QUANT) return launch_qa<0, true>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+      return SVDQ_ERR_INVALID_ARG;
+    case 16: return launch_qa<16, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 32: return launch_qa<32, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 48: return launch_qa<48, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 64: return launch_qa<64, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 80: return launch_qa<80, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 96: return launch_qa<96, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 112: return launch_qa<112, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 128: return launch_qa<128, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    default: return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  }
 }
 
 svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const uint8_t* Wq, const uint8_t* SFw,
                         float gs_w, const uint16_t* LAs, const uint16_t* L2p, int r, const uint16_t* bias, void* Y,
                         int y_fp32, int64_t M, int64_t N, int64_t K, int debug, uint64_t timeout_ns,
-                        cudaStream_t s) {
-  svdq_status st = check_shape(M, N, K, r);
+                        cudaStream_t s, int y_accum = 0) {
+  // y_accum: the rank-only mode (no 4-bit operands, K = 0) that adds the up-projection into Y.
+  svdq_status st = check_shape(M, N, y_accum ? 64 : K, r);
   if (st != SVDQ_OK) return st;
-  if (!Xq || !SFx || !Wq || !SFw || !Y || (r > 0 && (!LAs || !L2p)) || (y_fp32 != 0 && y_fp32 != 1))
+  if (y_accum ? (r == 0 || !LAs || !L2p || !Y || bias)
+              : (!Xq || !SFx || !Wq || !SFw || !Y || (r > 0 && (!LAs || !L2p))))
     return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(Xq) || !aligned16(SFx) || !aligned16(Wq) || !aligned16(SFw) || !aligned16(Y) ||
+  if (y_fp32 != 0 && y_fp32 != 1) return SVDQ_ERR_INVALID_ARG;
+  if ((!y_accum && (!aligned16(Xq) || !aligned16(SFx) || !aligned16(Wq) || !aligned16(SFw))) || !aligned16(Y) ||
       (bias && !aligned16(bias)) || (r > 0 && (!aligned16(LAs) || !aligned16(L2p))))
     return SVDQ_ERR_MISALIGNED;
   int dev;
@@ -151,31 +227,27 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
 
   CUtensorMap tm_xq, tm_wq, tm_las, tm_l2p;
-  if (!make_map_2d(&tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
-                   LN_BM) ||
-      !make_map_2d(&tm_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128,
-                   LN_BN / 2))
+  if (!y_accum &&
+      (!make_map_2d(&tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
+                    LN_BM) ||
+       !make_map_2d(&tm_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128,
+                    LN_BN / 2)))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
     if (!make_map_2d(&tm_las, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, LAs, (uint64_t)2 * r, (uint64_t)M,
                      (uint64_t)4 * r, 64, LN_BM) ||
-        !make_map_2d(&tm_l2p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2p, (uint64_t)2 * r, (uint64_t)N,
-                     (uint64_t)4 * r, 64, LN_BN / 2))
+        !make_map_2d(&tm_l2p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2p, (uint64_t)r, (uint64_t)N,
+                     (uint64_t)2 * r, 32, LN_BN / 2, CU_TENSOR_MAP_SWIZZLE_64B))
       return SVDQ_ERR_CUDA;
   } else {
     tm_las = tm_xq;
     tm_l2p = tm_wq;
   }
-  // The single-CTA kernel by default.  The CTA-pair kernel (256 x 256 tiles, half of B per CTA)
-  // gives the same results but measured slower on B200 (0.118 against 0.075 ms on the QKV layer):
-  // the signals between the two CTAs sit on every stage's critical path.  Debug bit 2 selects it.
-  const bool pair = (debug & LN_DBG_FORCE_PAIR) != 0;
-  if (pair && !d->linear_pair_attr) {
-    if (cudaFuncSetAttribute(k_linear_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, LP_SMEM) != cudaSuccess)
-      return SVDQ_ERR_CUDA;
-    d->linear_pair_attr = true;
+  if (y_accum) {                 // no K tiles: the 4-bit maps are never used
+    tm_xq = tm_las;
+    tm_wq = tm_l2p;
   }
-  if (!pair && !d->linear_attr) {
+  if (!d->linear_attr) {
     if (cudaFuncSetAttribute(k_linear, cudaFuncAttributeMaxDynamicSharedMemorySize, LN_SMEM) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     d->linear_attr = true;
@@ -187,22 +259,19 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   a.Y = Y;
   a.y_fp32 = y_fp32;
   a.y_vec32 = (reinterpret_cast<uintptr_t>(Y) & 31u) == 0 ? 1 : 0;
+  a.y_accum = y_accum;
   a.M = (int)M;
   a.N = (int)N;
-  a.K = (int)K;
+  a.K = y_accum ? 0 : (int)K;
   a.r = r;
   a.gs = gs_x * gs_w;
   a.debug = debug;
   a.timeout_ns = timeout_ns ? timeout_ns : LN_DEFAULT_TIMEOUT_NS;
-  if (pair) {
-    const int64_t tiles = ((M + LP_BM - 1) / LP_BM) * ((N + LP_BN - 1) / LP_BN);
-    const int64_t pairs = tiles < d->sms / 2 ? tiles : d->sms / 2;
-    k_linear_pair<<<(int)(2 * pairs), LP_THREADS, LP_SMEM, s>>>(tm_xq, tm_wq, tm_las, tm_l2p, a);
-  } else {
-    const int64_t tiles = ((M + LN_BM - 1) / LN_BM) * ((N + LN_BN - 1) / LN_BN);
-    const int grid = (int)(tiles < d->sms ? tiles : d->sms);
-    k_linear<<<grid, LN_THREADS, LN_SMEM, s>>>(tm_xq, tm_wq, tm_las, tm_l2p, a);
-  }
+  const int64_t tiles = ((M + LN_BM - 1) / LN_BM) * ((N + LN_BN - 1) / LN_BN);
+  const int grid = (int)(tiles < d->sms ? tiles : d->sms);
+  if (launch_pdl(k_linear, dim3(grid), dim3(LN_THREADS), (size_t)LN_SMEM, s, 1, tm_xq, tm_wq, tm_las, tm_l2p, a) !=
+      cudaSuccess)
+    return SVDQ_ERR_CUDA;
   return launch_status();
 }
 
@@ -231,7 +300,7 @@ size_t svdq_sf_bytes(int64_t rows, int64_t K) {
 }
 
 svdq_status svdq_pack_weight(const float* R, const uint16_t* L2b, int64_t K, int64_t N, int r, uint8_t* Wq,
-                             uint8_t* SFw, float* gs_w, uint16_t* L2p, svdq_stream_t stream) {
+                             uint8_t* SFw, float* gs_w, float* gs_w_host, uint16_t* L2p, svdq_stream_t stream) {
   svdq_status st = check_shape(1, N, K, r);
   if (st != SVDQ_OK) return st;
   if (!R || !Wq || !SFw || !gs_w || (r > 0 && (!L2b || !L2p))) return SVDQ_ERR_INVALID_ARG;
@@ -253,34 +322,69 @@ svdq_status svdq_pack_weight(const float* R, const uint16_t* L2b, int64_t K, int
   k_pack_weight<<<dim3((unsigned)(Npad / 128), (unsigned)(K / 64)), 128, 0, s>>>(R, (int)K, (int)N, (int)Npad, gs_w,
                                                                                   Wq, SFw);
   if (r > 0) k_layout_l2<<<(unsigned)((N + 127) / 128), 128, 0, s>>>(L2b, (int)N, r, L2p);
+  if ((st = launch_status()) != SVDQ_OK) return st;
+  if (gs_w_host) {
+    if (cudaMemcpyAsync(gs_w_host, gs_w, sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+svdq_status svdq_dequant_weight(const uint8_t* Wq, const uint8_t* SFw, const float* gs_w, int64_t K, int64_t N,
+                                float* Rq, svdq_stream_t stream) {
+  svdq_status st = check_shape(1, N, K, 0);
+  if (st != SVDQ_OK) return st;
+  if (!Wq || !SFw || !gs_w || !Rq) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(Wq) || !aligned16(SFw) || !aligned16(Rq)) return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  k_dequant_weight<<<dim3((unsigned)((N + 127) / 128), (unsigned)(K / 64)), 128, 0,
+                     reinterpret_cast<cudaStream_t>(stream)>>>(Wq, SFw, gs_w, (int)K, (int)N, Rq);
   return launch_status();
+}
+
+size_t svdq_quantize_act_workspace_bytes(int64_t M, int64_t K, int r) {
+  if (M < 1 || K < 64 || K % 64 != 0 || r < 0 || r % 16 != 0 || r > 128) return 0;
+  return qa_workspace_bytes(M, r);
 }
 
 svdq_status svdq_quantize_act(const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float gs_x,
                               const uint16_t* L1fT, int r, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
-                              svdq_stream_t stream) {
+                              void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
   svdq_status st = check_shape(M, 16, K, r);
   if (st != SVDQ_OK) return st;
   if (!X || !inv_s || !Xq || !SFx || (r > 0 && (!L1fT || !LAs))) return SVDQ_ERR_INVALID_ARG;
+  if (r > 0 && (!workspace || workspace_bytes < qa_workspace_bytes(M, r))) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(inv_s) || !aligned16(Xq) || !aligned16(SFx) ||
-      (r > 0 && (!aligned16(L1fT) || !aligned16(LAs))))
+      (r > 0 && (!aligned16(L1fT) || !aligned16(LAs) || !aligned16(workspace))))
     return SVDQ_ERR_MISALIGNED;
   int dev;
   DevInfo* d;
   if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  switch (r) {
-    case 0: return launch_qa<0>(d, 0, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    case 16: return launch_qa<16>(d, 1, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    case 32: return launch_qa<32>(d, 2, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    case 48: return launch_qa<48>(d, 3, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    case 64: return launch_qa<64>(d, 4, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    case 80: return launch_qa<80>(d, 5, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    case 96: return launch_qa<96>(d, 6, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    case 112: return launch_qa<112>(d, 7, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    case 128: return launch_qa<128>(d, 8, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, s);
-    default: return SVDQ_ERR_UNSUPPORTED_SHAPE;
-  }
+  return dispatch_qa<true>(d, r, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, workspace,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_lowrank_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* L1fT, int r, float lr_scale,
+                              uint16_t* LAs, void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
+  svdq_status st = check_shape(M, 16, K, r);
+  if (st != SVDQ_OK) return st;
+  if (r == 0 || !X || !L1fT || !LAs || !workspace || workspace_bytes < qa_workspace_bytes(M, r))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(L1fT) || !aligned16(LAs) || !aligned16(workspace)) return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  return dispatch_qa<false>(d, r, X, M, K, nullptr, 1.0f, L1fT, lr_scale, nullptr, nullptr, LAs, workspace,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_lowrank_up(const uint16_t* LAs, const uint16_t* L2p, int r, float gs, void* Y, int y_fp32,
+                            int64_t M, int64_t N, svdq_stream_t stream) {
+  return linear_impl(nullptr, nullptr, 1.0f, nullptr, nullptr, gs, LAs, L2p, r, nullptr, Y, y_fp32, M, N, 0, 0, 0,
+                     reinterpret_cast<cudaStream_t>(stream), 1);
 }
 
 svdq_status svdq_linear(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const uint8_t* Wq, const uint8_t* SFw,
@@ -294,9 +398,7 @@ svdq_status svdq_linear_debug(const uint8_t* Xq, const uint8_t* SFx, float gs_x,
                               const uint8_t* SFw, float gs_w, const uint16_t* LAs, const uint16_t* L2p, int r,
                               const uint16_t* bias, void* Y, int y_fp32, int64_t M, int64_t N, int64_t K,
                               int debug_flags, uint64_t timeout_ns, svdq_stream_t stream) {
-  if ((debug_flags & ~(LN_DBG_NO_LOADS | LN_DBG_FORCE_SINGLE | LN_DBG_FORCE_PAIR)) ||
-      ((debug_flags & LN_DBG_FORCE_SINGLE) && (debug_flags & LN_DBG_FORCE_PAIR)))
-    return SVDQ_ERR_INVALID_ARG;
+  if (debug_flags & ~LN_DBG_NO_LOADS) return SVDQ_ERR_INVALID_ARG;
   return linear_impl(Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p, r, bias, Y, y_fp32, M, N, K, debug_flags, timeout_ns,
                      reinterpret_cast<cudaStream_t>(stream));
 }

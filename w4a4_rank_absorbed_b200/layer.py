@@ -25,6 +25,18 @@ def _f32(x) -> float:
     return float(np.float32(x))
 
 
+def check_device(t: Optional[torch.Tensor], device: torch.device, name: str) -> None:
+    """Raise ValueError unless tensor `t` (when given) lives on `device`.
+
+    The library launches on the calling thread's current device with raw pointers; a tensor on
+    another GPU would be read through a pointer that device cannot resolve."""
+    if t is None:
+        return
+    want = torch.device(device)
+    if t.device.type != want.type or (want.index is not None and t.device.index != want.index):
+        raise ValueError(f"{name} is on {t.device}, the layer on {want}")
+
+
 class SVDQLinear:
     def __init__(self, data: LayerData, device: Optional[torch.device] = None, stream=None):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
@@ -38,9 +50,17 @@ class SVDQLinear:
             self.Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
             self.SFw = torch.empty(_C.svdq_sf_bytes(N, K), dtype=torch.uint8, device=dev)
             self.gs_w_dev = torch.empty(1, dtype=torch.float32, device=dev)
-            self.L2p = torch.empty((N, 2 * r), dtype=torch.bfloat16, device=dev) if r else None
-            _C.svdq_pack_weight(R, L2b, K, N, r, self.Wq, self.SFw, self.gs_w_dev, self.L2p, stream)
-            self.gs_w = _f32(self.gs_w_dev.item())     # synchronises the stream
+            self.L2p = torch.empty((N, r), dtype=torch.bfloat16, device=dev) if r else None
+            # The packing stream may differ from torch's current stream: the staging tensors are
+            # produced on the current stream, so the packing waits for it; the library writes gs_w
+            # to host memory after synchronising the packing stream, so R and L2b are no longer
+            # read when they are freed below.
+            if stream is not None:
+                ps = stream if isinstance(stream, torch.cuda.Stream) else \
+                    torch.cuda.ExternalStream(_C.stream_handle(stream), device=dev)
+                ps.wait_stream(torch.cuda.current_stream(dev))
+            self.gs_w = _f32(_C.svdq_pack_weight(R, L2b, K, N, r, self.Wq, self.SFw, self.gs_w_dev, self.L2p,
+                                                 stream, sync=True))
             del R, L2b
             self.inv_s = data.inv_s.to(dev, torch.float32).contiguous()
             self.L1fT = data.L1fT.to(dev).contiguous() if r else None
@@ -49,25 +69,35 @@ class SVDQLinear:
         self._act: Dict[int, tuple] = {}
 
     def act_buffers(self, M: int):
-        """Device buffers of the quantized activations for M rows (allocated once per M)."""
+        """Device buffers of the quantized activations for M rows (allocated once per M): Xq, SFx, LAs."""
+        return self._act_set(M)[:3]
+
+    def _act_set(self, M: int):
         if M not in self._act:
             K, r, dev = self.K, self.r, self.device
-            self._act[M] = (torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
-                            torch.empty(_C.svdq_sf_bytes(M, K), dtype=torch.uint8, device=dev),
-                            torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev) if r else None)
+            with torch.cuda.device(dev):
+                self._act[M] = (torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                                torch.empty(_C.svdq_sf_bytes(M, K), dtype=torch.uint8, device=dev),
+                                torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev) if r else None,
+                                _C.new_workspace(M, K, r, dev))
         return self._act[M]
 
     def quantize(self, X: torch.Tensor, stream=None):
+        check_device(X, self.device, "X")
         M = X.shape[0]
-        Xq, SFx, LAs = self.act_buffers(M)
-        _C.svdq_quantize_act(X, M, self.K, self.inv_s, self.gs_x, self.L1fT, self.r, self.lr_scale,
-                             Xq, SFx, LAs, stream)
+        Xq, SFx, LAs, ws = self._act_set(M)
+        with torch.cuda.device(self.device):
+            _C.svdq_quantize_act(X, M, self.K, self.inv_s, self.gs_x, self.L1fT, self.r, self.lr_scale,
+                                 Xq, SFx, LAs, ws, stream)
         return Xq, SFx, LAs
 
     def gemm(self, Xq, SFx, LAs, Y: torch.Tensor, stream=None):
+        for t, name in ((Xq, "Xq"), (SFx, "SFx"), (LAs, "LAs"), (Y, "Y")):
+            check_device(t, self.device, name)
         M = Xq.shape[0]
-        _C.svdq_linear(Xq, SFx, self.gs_x, self.Wq, self.SFw, self.gs_w, LAs, self.L2p, self.r, self.bias,
-                       Y, 1 if Y.dtype == torch.float32 else 0, M, self.N, self.K, stream)
+        with torch.cuda.device(self.device):
+            _C.svdq_linear(Xq, SFx, self.gs_x, self.Wq, self.SFw, self.gs_w, LAs, self.L2p, self.r, self.bias,
+                           Y, 1 if Y.dtype == torch.float32 else 0, M, self.N, self.K, stream)
         return Y
 
     def forward(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, y_fp32: bool = False,
@@ -75,6 +105,8 @@ class SVDQLinear:
         """Y = layer(X); X bf16 [M, K] on the device; returns bf16 (or fp32) [M, N]."""
         if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != self.K:
             raise ValueError("X must be bf16 [M, K]")
+        check_device(X, self.device, "X")
+        check_device(out, self.device, "out")
         M = X.shape[0]
         if out is None:
             out = torch.empty((M, self.N), dtype=torch.float32 if y_fp32 else torch.bfloat16, device=self.device)

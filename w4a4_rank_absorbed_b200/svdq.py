@@ -26,7 +26,8 @@ SVDQ_ERR_TIMEOUT = 5
 SVDQ_ERR_DEVICE = 6
 
 EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_weight", "svdq_quantize_act",
-            "svdq_linear", "svdq_get_device_error", "svdq_linear_debug")
+            "svdq_linear", "svdq_lowrank_down", "svdq_lowrank_up", "svdq_get_device_error", "svdq_linear_debug",
+            "svdq_quantize_act_workspace_bytes", "svdq_dequant_weight")
 
 
 class SVDQError(RuntimeError):
@@ -58,14 +59,22 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_sf_bytes.restype = ctypes.c_size_t
     lib.svdq_sf_bytes.argtypes = [_I64, _I64]
     lib.svdq_pack_weight.restype = _I
-    lib.svdq_pack_weight.argtypes = [_P, _P, _I64, _I64, _I, _P, _P, _P, _P, _P]
+    lib.svdq_pack_weight.argtypes = [_P, _P, _I64, _I64, _I, _P, _P, _P, ctypes.POINTER(_F), _P, _P]
     lib.svdq_quantize_act.restype = _I
-    lib.svdq_quantize_act.argtypes = [_P, _I64, _I64, _P, _F, _P, _I, _F, _P, _P, _P, _P]
+    lib.svdq_quantize_act.argtypes = [_P, _I64, _I64, _P, _F, _P, _I, _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.svdq_quantize_act_workspace_bytes.restype = ctypes.c_size_t
+    lib.svdq_quantize_act_workspace_bytes.argtypes = [_I64, _I64, _I]
     lib.svdq_linear.restype = _I
     lib.svdq_linear.argtypes = [_P, _P, _F, _P, _P, _F, _P, _P, _I, _P, _P, _I, _I64, _I64, _I64, _P]
     lib.svdq_linear_debug.restype = _I
     lib.svdq_linear_debug.argtypes = [_P, _P, _F, _P, _P, _F, _P, _P, _I, _P, _P, _I, _I64, _I64, _I64, _I,
                                       ctypes.c_uint64, _P]
+    lib.svdq_dequant_weight.restype = _I
+    lib.svdq_dequant_weight.argtypes = [_P, _P, _P, _I64, _I64, _P, _P]
+    lib.svdq_lowrank_down.restype = _I
+    lib.svdq_lowrank_down.argtypes = [_P, _I64, _I64, _P, _I, _F, _P, _P, ctypes.c_size_t, _P]
+    lib.svdq_lowrank_up.restype = _I
+    lib.svdq_lowrank_up.argtypes = [_P, _P, _I, _F, _P, _I, _I64, _I64, _P]
     lib.svdq_get_device_error.restype = _I
     lib.svdq_get_device_error.argtypes = [_P, ctypes.POINTER(_I)]
     _lib = lib
@@ -93,6 +102,13 @@ def _ptr(t: Optional[torch.Tensor], dtype=None, name: str = "") -> Optional[int]
     return t.data_ptr()
 
 
+def stream_handle(stream) -> int:
+    """The cudaStream_t handle (as an int) of a torch stream or a raw handle."""
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -114,20 +130,41 @@ def svdq_version() -> int:
     return int(load_library().svdq_version())
 
 
-def svdq_pack_weight(R, L2b, K, N, r, Wq, SFw, gs_w, L2p, stream=None) -> None:
+def svdq_pack_weight(R, L2b, K, N, r, Wq, SFw, gs_w, L2p, stream=None, sync: bool = True) -> Optional[float]:
+    """Packs the residual weight.  With sync=True (the default) the call synchronises the stream and
+    returns gs_w as a Python float (the library writes it to host memory); with sync=False it stays
+    asynchronous and returns None (gs_w is then only in the device tensor)."""
     lib = load_library()
+    host = _F(0.0)
     st = lib.svdq_pack_weight(_ptr(R, torch.float32, "R"), _ptr(L2b, torch.bfloat16, "L2b"), K, N, r,
                               _ptr(Wq, torch.uint8, "Wq"), _ptr(SFw, torch.uint8, "SFw"),
-                              _ptr(gs_w, torch.float32, "gs_w"), _ptr(L2p, torch.bfloat16, "L2p"), _stream(stream))
+                              _ptr(gs_w, torch.float32, "gs_w"), ctypes.byref(host) if sync else None,
+                              _ptr(L2p, torch.bfloat16, "L2p"), _stream(stream))
     _check(st, "svdq_pack_weight")
+    return float(host.value) if sync else None
 
 
-def svdq_quantize_act(X, M, K, inv_s, gs_x, L1fT, r, lr_scale, Xq, SFx, LAs, stream=None) -> None:
+def svdq_quantize_act_workspace_bytes(M: int, K: int, r: int) -> int:
+    return int(load_library().svdq_quantize_act_workspace_bytes(M, K, r))
+
+
+def new_workspace(M: int, K: int, r: int, device=None) -> Optional[torch.Tensor]:
+    """A zero-filled workspace for svdq_quantize_act / svdq_lowrank_down (None when none is needed)."""
+    n = svdq_quantize_act_workspace_bytes(M, K, r)
+    return torch.zeros(n, dtype=torch.uint8, device=device if device is not None else "cuda") if n else None
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def svdq_quantize_act(X, M, K, inv_s, gs_x, L1fT, r, lr_scale, Xq, SFx, LAs, workspace=None, stream=None) -> None:
     lib = load_library()
     st = lib.svdq_quantize_act(_ptr(X, torch.bfloat16, "X"), M, K, _ptr(inv_s, torch.float32, "inv_s"),
                                float(gs_x), _ptr(L1fT, torch.bfloat16, "L1fT"), r, float(lr_scale),
                                _ptr(Xq, torch.uint8, "Xq"), _ptr(SFx, torch.uint8, "SFx"),
-                               _ptr(LAs, torch.bfloat16, "LAs"), _stream(stream))
+                               _ptr(LAs, torch.bfloat16, "LAs"), _ptr(workspace, torch.uint8, "workspace"),
+                               _nbytes(workspace), _stream(stream))
     _check(st, "svdq_quantize_act")
 
 
@@ -150,6 +187,29 @@ def svdq_linear_debug(Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p, r, bias, Y, y_fp32
                                _ptr(bias, torch.bfloat16, "bias"), _ptr(Y, (torch.bfloat16, torch.float32), "Y"),
                                int(y_fp32), M, N, K, int(debug_flags), int(timeout_ns), _stream(stream))
     _check(st, "svdq_linear_debug")
+
+
+def svdq_dequant_weight(Wq, SFw, gs_w, K, N, Rq, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_dequant_weight(_ptr(Wq, torch.uint8, "Wq"), _ptr(SFw, torch.uint8, "SFw"),
+                                 _ptr(gs_w, torch.float32, "gs_w"), K, N, _ptr(Rq, torch.float32, "Rq"),
+                                 _stream(stream))
+    _check(st, "svdq_dequant_weight")
+
+
+def svdq_lowrank_down(X, M, K, L1fT, r, lr_scale, LAs, workspace, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_lowrank_down(_ptr(X, torch.bfloat16, "X"), M, K, _ptr(L1fT, torch.bfloat16, "L1fT"), r,
+                               float(lr_scale), _ptr(LAs, torch.bfloat16, "LAs"),
+                               _ptr(workspace, torch.uint8, "workspace"), _nbytes(workspace), _stream(stream))
+    _check(st, "svdq_lowrank_down")
+
+
+def svdq_lowrank_up(LAs, L2p, r, gs, Y, y_fp32, M, N, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_lowrank_up(_ptr(LAs, torch.bfloat16, "LAs"), _ptr(L2p, torch.bfloat16, "L2p"), r, float(gs),
+                             _ptr(Y, (torch.bfloat16, torch.float32), "Y"), int(y_fp32), M, N, _stream(stream))
+    _check(st, "svdq_lowrank_up")
 
 
 def svdq_get_device_error(stream=None):
