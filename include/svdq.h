@@ -75,7 +75,8 @@ typedef enum {
     SVDQ_ERR_MISALIGNED = 3,         /* a pointer not 16-byte aligned                  */
     SVDQ_ERR_CUDA = 4,               /* a CUDA runtime/driver call or launch failed    */
     SVDQ_ERR_TIMEOUT = 5,            /* a kernel's bounded wait ran out (device error) */
-    SVDQ_ERR_DEVICE = 6              /* current device is not compute capability 10.x  */
+    SVDQ_ERR_DEVICE = 6,             /* current device is not compute capability 10.x  */
+    SVDQ_ERR_SCRATCH = 7             /* shape needs more than the library's own scratch */
 } svdq_status;
 
 /* Human-readable name of a status code (static string). */
@@ -170,6 +171,37 @@ SVDQ_API svdq_status svdq_quantize_act(const uint16_t* X, int64_t M, int64_t K, 
 /* Bytes of the workspace svdq_quantize_act and svdq_lowrank_down need for M rows of K columns at
  * rank r (0 when r == 0; 0 for a shape the calls reject).  Independent of the device. */
 SVDQ_API size_t svdq_quantize_act_workspace_bytes(int64_t M, int64_t K, int r);
+
+/*
+ * svdq_quantize_act_noalloc -- svdq_quantize_act for callers that cannot
+ * allocate device memory.  (The pages have no counterpart: this is an entry
+ * point of the library, not a step of the method.)
+ *
+ * Some callers have no way to obtain a workspace: a host application whose
+ * memory pool owns all of the device memory and forbids other allocations, or
+ * a runtime that must not allocate once it is running (cudaMalloc can
+ * synchronise the device and takes an unbounded time).  This entry point takes
+ * the same arguments as svdq_quantize_act minus the workspace and allocates
+ * nothing: the partial sums of the K-split down-projection live in a scratch
+ * array the library declares in device memory, SVDQ_NOALLOC_SCRATCH_BYTES
+ * (8 MiB) on every GPU that loads the library, held until the process exits.
+ *
+ *   - A shape whose K-split needs more than that (about 8 MiB of partial sums
+ *     plus one counter per 128 rows; e.g. M = 4608, r = 32 needs 2.4 MiB) is
+ *     refused with SVDQ_ERR_SCRATCH before anything is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - Every call on a device shares the one array.  Each call clears the
+ *     counters it needs (an asynchronous memset on `stream`); calls whose
+ *     kernels overlap on the GPU (different streams, or graphs replayed
+ *     concurrently) race on the array and give undefined LAs.
+ *   - Results are identical to svdq_quantize_act's.
+ */
+#define SVDQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+SVDQ_API svdq_status svdq_quantize_act_noalloc(const uint16_t* X, int64_t M, int64_t K, const float* inv_s,
+                              float gs_x, const uint16_t* L1fT, int r, float lr_scale,
+                              uint8_t* Xq, uint8_t* SFx, uint16_t* LAs, svdq_stream_t stream);
 
 /*
  * svdq_linear -- block-scaled NVFP4 GEMM on the tcgen05 tensor cores with the

@@ -152,6 +152,32 @@ size_t qa_workspace_bytes(int64_t M, int r) {
   return r > 0 ? qa_ticket_bytes(M) + (size_t)QB_MAX_SPLIT * (size_t)pad128(M) * (size_t)r * 4 : 0;
 }
 
+// ------------------------------------------------ scratch of svdq_quantize_act_noalloc ---
+// Device memory the library owns for callers that cannot allocate: the counters and partial sums
+// of kernel 2's K split.  In host code the name stands for a host-side handle, not a device address,
+// so the kernels are given the address cudaGetSymbolAddress returns for the current device.
+constexpr size_t kNoAllocScratchBytes = SVDQ_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Bytes of the scratch a call uses: the counters, then the partial sums of the split the launch takes.
+size_t noalloc_scratch_need(int64_t M, int64_t K, int r, int sms) {
+  return qa_ticket_bytes(M) + (size_t)qa_split(M, K, sms) * (size_t)pad128(M) * (size_t)r * 4;
+}
+
+// Device address of the scratch array on device `dev` (the current device), looked up once.
+svdq_status noalloc_scratch(int dev, DevInfo* d, void** out) {
+  (void)d;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SVDQ_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SVDQ_OK;
+}
+
 template <int R, bool QUANT>
 svdq_status launch_qa(DevInfo* d, const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float gs_x,
                       const uint16_t* L1fT, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
@@ -288,6 +314,7 @@ const char* svdq_status_string(int status) {
     case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA";
     case SVDQ_ERR_TIMEOUT: return "SVDQ_ERR_TIMEOUT";
     case SVDQ_ERR_DEVICE: return "SVDQ_ERR_DEVICE";
+    case SVDQ_ERR_SCRATCH: return "SVDQ_ERR_SCRATCH";
     default: return "SVDQ_ERR_UNKNOWN";
   }
 }
@@ -365,6 +392,29 @@ svdq_status svdq_quantize_act(const uint16_t* X, int64_t M, int64_t K, const flo
   if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
   return dispatch_qa<true>(d, r, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, workspace,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_quantize_act_noalloc(const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float gs_x,
+                                      const uint16_t* L1fT, int r, float lr_scale, uint8_t* Xq, uint8_t* SFx,
+                                      uint16_t* LAs, svdq_stream_t stream) {
+  svdq_status st = check_shape(M, 16, K, r);
+  if (st != SVDQ_OK) return st;
+  if (!X || !inv_s || !Xq || !SFx || (r > 0 && (!L1fT || !LAs))) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(inv_s) || !aligned16(Xq) || !aligned16(SFx) ||
+      (r > 0 && (!aligned16(L1fT) || !aligned16(LAs))))
+    return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  if (r > 0) {
+    if (noalloc_scratch_need(M, K, r, d->sms) > kNoAllocScratchBytes) return SVDQ_ERR_SCRATCH;
+    if ((st = noalloc_scratch(dev, d, &ws)) != SVDQ_OK) return st;
+    // the row-block counters start at 0 (a call that ran out of time can leave them set)
+    if (cudaMemsetAsync(ws, 0, qa_ticket_bytes(M), s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  }
+  return dispatch_qa<true>(d, r, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
 }
 
 svdq_status svdq_lowrank_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* L1fT, int r, float lr_scale,

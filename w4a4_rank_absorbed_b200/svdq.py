@@ -24,10 +24,11 @@ SVDQ_ERR_MISALIGNED = 3
 SVDQ_ERR_CUDA = 4
 SVDQ_ERR_TIMEOUT = 5
 SVDQ_ERR_DEVICE = 6
+SVDQ_ERR_SCRATCH = 7
 
 EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_weight", "svdq_quantize_act",
             "svdq_linear", "svdq_lowrank_down", "svdq_lowrank_up", "svdq_get_device_error", "svdq_linear_debug",
-            "svdq_quantize_act_workspace_bytes", "svdq_dequant_weight")
+            "svdq_quantize_act_workspace_bytes", "svdq_dequant_weight", "svdq_quantize_act_noalloc")
 
 
 class SVDQError(RuntimeError):
@@ -62,6 +63,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_pack_weight.argtypes = [_P, _P, _I64, _I64, _I, _P, _P, _P, ctypes.POINTER(_F), _P, _P]
     lib.svdq_quantize_act.restype = _I
     lib.svdq_quantize_act.argtypes = [_P, _I64, _I64, _P, _F, _P, _I, _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.svdq_quantize_act_noalloc.restype = _I
+    lib.svdq_quantize_act_noalloc.argtypes = [_P, _I64, _I64, _P, _F, _P, _I, _F, _P, _P, _P, _P]
     lib.svdq_quantize_act_workspace_bytes.restype = ctypes.c_size_t
     lib.svdq_quantize_act_workspace_bytes.argtypes = [_I64, _I64, _I]
     lib.svdq_linear.restype = _I
@@ -142,6 +145,17 @@ def svdq_pack_weight(R, L2b, K, N, r, Wq, SFw, gs_w, L2p, stream=None, sync: boo
                               _ptr(L2p, torch.bfloat16, "L2p"), _stream(stream))
     _check(st, "svdq_pack_weight")
     return float(host.value) if sync else None
+
+
+def svdq_quantize_act_noalloc(X, M, K, inv_s, gs_x, L1fT, r, lr_scale, Xq, SFx, LAs, stream=None) -> None:
+    """svdq_quantize_act without a workspace: the library's own device scratch holds the partial sums
+    (for callers that cannot allocate device memory; see include/svdq.h for the size limit)."""
+    lib = load_library()
+    st = lib.svdq_quantize_act_noalloc(_ptr(X, torch.bfloat16, "X"), M, K, _ptr(inv_s, torch.float32, "inv_s"),
+                                       float(gs_x), _ptr(L1fT, torch.bfloat16, "L1fT"), r, float(lr_scale),
+                                       _ptr(Xq, torch.uint8, "Xq"), _ptr(SFx, torch.uint8, "SFx"),
+                                       _ptr(LAs, torch.bfloat16, "LAs"), _stream(stream))
+    _check(st, "svdq_quantize_act_noalloc")
 
 
 def svdq_quantize_act_workspace_bytes(M: int, K: int, r: int) -> int:
