@@ -104,6 +104,40 @@ SVDQ_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, vol
   }
 }
 
+// Non-blocking test of the phase with parity `parity`.
+SVDQ_DEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for the single threads on a pipeline's critical path (copy producers, MMA issuers):
+// polls with the non-blocking test, so the thread sees the phase complete without the wake-up
+// delay a suspended try_wait can add.  Same time-out and abort behaviour as mbar_wait.
+SVDQ_DEV bool mbar_wait_spin(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, volatile int* abort,
+                             unsigned site) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 0;; ++n) {
+    if (mbar_test_wait(a, parity)) return true;
+    if ((n & 15u) == 15u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        *abort = 1;
+        report_timeout(site);
+        return false;
+      }
+    }
+  }
+}
+
 // mbar_wait for a barrier that also receives arrivals released at cluster scope by the other
 // CTA of a pair: the successful test acquires at cluster scope.
 SVDQ_DEV bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
@@ -144,6 +178,14 @@ SVDQ_DEV void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       ::"r"(smem_u32(dst)), "l"(m), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 3-D tiled load: box at (x, y, z) into shared memory, completion counted in bytes on `bar`.
+SVDQ_DEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(smem_u32(dst)), "l"(m), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
           const int stage = gidx % LN_STAGES;
           const uint32_t phase = (uint32_t)((gidx / LN_STAGES) & 1);
           int free_slot = 1;
-          if (lane == 0) free_slot = mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag, 0x301) ? 1 : 0;
+          if (lane == 0) free_slot = mbar_wait_spin(&empty[stage], phase ^ 1u, tmo, abort_flag, 0x301) ? 1 : 0;
           if (!__shfl_sync(0xffffffffu, free_slot, 0)) { ok = false; break; }
           const bool mine = loader && g == stage;
           const unsigned smask = 7u << (LN_STREAMS * stage);   // the stage's three lanes
@@ -340,11 +340,11 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        if (it > 0 && !mbar_wait(acc_empty, (uint32_t)((it - 1) & 1), tmo, abort_flag, 0x311)) break;
+        if (it > 0 && !mbar_wait_spin(acc_empty, (uint32_t)((it - 1) & 1), tmo, abort_flag, 0x311)) break;
         tc_fence_after();
         for (int kt = 0; kt < nst; ++kt) {
-          if (!mbar_wait(&full[stage], phase, tmo, abort_flag, 0x312) ||
-              !mbar_wait(&sf_ready[stage], phase, tmo, abort_flag, 0x314)) {
+          if (!mbar_wait_spin(&full[stage], phase, tmo, abort_flag, 0x312) ||
+              !mbar_wait_spin(&sf_ready[stage], phase, tmo, abort_flag, 0x314)) {
             ok = false;
             break;
           }

@@ -11,20 +11,29 @@
 //
 // Work split: a CTA owns 128 rows and a contiguous range of the K axis; `split`
 // CTAs share a row block (split = 1 when there are enough row blocks to fill
-// the GPU).  The K axis is read in 64-column chunks through an S-stage ring
-// (TMA, 128-byte swizzle): the 128 x 64 X box, the r x 64 L1f^T box and the
-// chunk's 64 smoothing factors.  Roles (18 warps):
-//   warp 0      producer: three lanes issue a stage's three copies in one
-//               converged instruction; the lanes rotate with the ring slot so no
-//               thread has two copies of one stream in flight.
-//   warp 1      TMEM owner and MMA issuer (one thread): per chunk four
-//               tcgen05.mma.kind::f16 of 128 x r x 16 (A = the X box, B = the
-//               L1f^T box) into one fp32 accumulator of r TMEM columns; each
-//               chunk's commit is one of the arrivals that frees its stage.
-//   warps 2-17  quantizers: thread i takes row i / 4, group i % 4 of the chunk
-//               (16 values), writes 8 bytes of codes and, gathered over the
-//               row's four lanes, one 32-bit word of scales.
-// After the last chunk, four of the quantizer warps (one per TMEM lane quarter)
+// the GPU).  The K axis is read in stages of two 64-column chunks through an
+// S-stage ring: one 3-D TMA box (dims: 64 columns, rows, K/64 chunks) brings
+// both chunks of all 128 rows, landing as two 128-byte-swizzled 128-row tiles
+// (the reads are 256 contiguous bytes a row, which streams from HBM faster than
+// 128-byte pieces), and one more box the matching r x 64 L1f^T tiles.  A copy
+// instruction holds its warp for a few hundred nanoseconds, so each stream has
+// a producer warp of its own and a stage takes one instruction per stream; the
+// smoothing factors (a few KB, L1-resident) are read by the quantizers
+// directly.  Roles (19 warps):
+//   warp 0      X producer, warp 18 L1f^T producer (one lane each).
+//   warp 1      TMEM owner and MMA issuer (one thread): per stage eight
+//               tcgen05.mma.kind::f16 of 128 x r x 16 (A = an X tile, B = the
+//               chunk's L1f^T tile) into one fp32 accumulator of r TMEM columns;
+//               each stage's commit is one of the arrivals that frees it.
+//   warps 2-17  quantizers: thread i takes group i % 4 of chunk (i / 8) % 2 of
+//               the stage for rows 2 (i / 16) + (i / 4) % 2 and that row + 64: two
+//               independent groups of 16 values (two chains of work in flight)
+//               that share their 16 smoothing factors.  A quarter-warp so reads
+//               rows r and r ^ 1 of one chunk, whose 128-byte swizzle patterns
+//               are complementary: its eight 16-byte reads hit eight different
+//               bank groups.  Each group gives 8 bytes of codes and, gathered
+//               over the four lanes of a row and chunk, one 32-bit word of scales.
+// After the last stage, four of the quantizer warps (one per TMEM lane quarter)
 // read the accumulator.  With split = 1 it goes through shared memory straight
 // to LAs.  Otherwise each CTA writes its partial sums to the caller's workspace
 // and takes a ticket for its row block; the CTA that takes the last ticket adds
@@ -45,22 +54,25 @@ constexpr int QB_ROWS = 128;
 constexpr int QB_CHUNK = 64;                 // bf16 columns per chunk (128 bytes)
 constexpr int QB_QWARPS = 16;
 constexpr int QB_WARP_Q0 = 2;                // first quantizer warp
-constexpr int QB_THREADS = (QB_WARP_Q0 + QB_QWARPS) * 32;
+constexpr int QB_WARP_L1 = QB_WARP_Q0 + QB_QWARPS;   // producer of the L1f^T tiles
+constexpr int QB_THREADS = (QB_WARP_L1 + 1) * 32;
 constexpr int QB_MAX_SPLIT = 8;                // power of two: 128 rows / split, ticket arithmetic
 constexpr int QB_RING_BYTES = 200 * 1024;
 constexpr int QB_MAX_STAGES = 12;
 
 template <int R>
 struct QbCfg {
-  static constexpr int kXBytes = QB_ROWS * 128;
-  static constexpr int kLBytes = R * 128;
-  static constexpr int kInvBytes = 1024;     // 64 floats used; keeps the next stage 1024-aligned
-  static constexpr int kStageBytes = kXBytes + kLBytes + kInvBytes;
+  static constexpr int kChunks = 2;                              // 64-column chunks per stage
+  static constexpr int kXTile = QB_ROWS * 128;                   // one chunk of 128 rows
+  static constexpr int kLTile = R * 128;                         // one chunk of L1f^T
+  static constexpr int kXBytes = kChunks * kXTile;
+  static constexpr int kLBytes = kChunks * kLTile;
+  static constexpr int kStageBytes = kXBytes + kLBytes;
   static constexpr int kStages = QB_RING_BYTES / kStageBytes < QB_MAX_STAGES ? QB_RING_BYTES / kStageBytes
                                                                              : QB_MAX_STAGES;
   static constexpr int kRingBytes = kStages * kStageBytes;
-  static_assert(QB_ROWS * R * 4 <= kRingBytes, "the reduction buffer reuses the ring");
-  static_assert(QB_ROWS * R * 4 + 16 <= kRingBytes, "the last-CTA flag sits after it");
+  static_assert(QB_ROWS * R * 4 + 16 <= kRingBytes, "the reduction buffer and last-CTA flag reuse the ring");
+  static_assert(kStages >= 2, "ring");
   static constexpr int kRcpOff = kRingBytes;                // 128-entry 1/d table
   static constexpr int kBarOff = kRcpOff + 128 * 4;
   static constexpr int kSmem = kBarOff + (2 * kStages + 2) * 8 + 16 + 1024;
@@ -120,8 +132,10 @@ SVDQ_DEV bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, vol
 
 template <int R, bool QUANT>
 __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
-    const __grid_constant__ CUtensorMap tm_x,   // bf16 {K, M}, box {64, 128}, 128B swizzle
-    const __grid_constant__ CUtensorMap tm_l1,  // bf16 {K, R}, box {64, R}, 128B swizzle
+    const __grid_constant__ CUtensorMap tm_x,   // bf16 {64, M, K/64} (strides 2K, 128 bytes), box {64, 128, 2}, SW128
+    const __grid_constant__ CUtensorMap tm_l1,  // bf16 {64, R, K/64} (strides 2K, 128 bytes), box {64, R, 2}, SW128
+    const __grid_constant__ CUtensorMap tm_x1,  // bf16 {K, M}, box {64, 128}, SW128: a lone last chunk
+    const __grid_constant__ CUtensorMap tm_l11, // bf16 {K, R}, box {64, R}, SW128: a lone last chunk
     const float* __restrict__ inv_s, float gs_x, float lr_scale, int M, int K, int Mpad, int split,
     uint8_t* __restrict__ Xq, uint8_t* __restrict__ SFx, uint16_t* __restrict__ LAs,
     float* __restrict__ ws_part,            // split > 1: [split][Mpad][R] partial sums
@@ -145,13 +159,14 @@ __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
   const int rb = (int)(blockIdx.x / (unsigned)split);
   const int m0 = rb * QB_ROWS;
   const int nch = K / QB_CHUNK;
-  const int c_begin = rank * nch / split;
-  const int my = (rank + 1) * nch / split - c_begin;       // chunks of this CTA (>= 1)
+  const int nunits = (nch + 1) >> 1;                          // stages of two chunks (the last may hold one)
+  const int u_begin = rank * nunits / split;
+  const int my = (rank + 1) * nunits / split - u_begin;       // stages of this CTA (>= 1)
   const uint64_t tmo = timeout_ns;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], R > 0 ? 2 : 1);      // one expect-tx arrival per producer
       mbar_init(&empty[s], QB_QWARPS + (R > 0 ? 1 : 0));
     }
     mbar_init(acc_full, 1);
@@ -172,7 +187,11 @@ __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
-    if (R > 0) tma_prefetch_desc(&tm_l1);
+    tma_prefetch_desc(&tm_x1);
+    if (R > 0) {
+      tma_prefetch_desc(&tm_l1);
+      tma_prefetch_desc(&tm_l11);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -182,38 +201,41 @@ __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
   griddep_wait();
   griddep_launch_dependents();
 
-  if (warp == 0) {
-    // ------------------------------------------------------------- producer --
-    const int k = lane % 3;
-    int issued = 0;
-    bool ok = true;
-    for (int i = 0; i < my; ++i) {
-      const int s = i % S;
-      if (i >= S && !warp_wait(&empty[s], (uint32_t)(((i / S) - 1) & 1), tmo, abort_flag, 0x201)) {
-        ok = false;
-        break;
-      }
-      const int g = s % 10;                   // lanes 3g .. 3g + 2 serve slot s
-      if (lane >= 3 * g && lane < 3 * g + 3) {
+  if (warp == 0 || warp == QB_WARP_L1) {
+    // ------------------------------------------------------------ producers --
+    // Warp 0 fetches the X tiles, warp 18 the L1f^T tiles (r > 0), each with one lane.  With an odd
+    // number of chunks the last stage holds one: it is fetched with the 2-D maps, so no copy reaches
+    // past the last chunk of K.
+    const bool xw = warp == 0;
+    if (lane == 0 && (xw || R > 0)) {
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < my; ++i) {
+        const int s = i % S;
+        if (i >= S && !mbar_wait_spin(&empty[s], (uint32_t)(((i / S) - 1) & 1), tmo, abort_flag, 0x201)) {
+          ok = false;
+          break;
+        }
         uint8_t* st = smem + s * Cfg::kStageBytes;
-        const int c = c_begin + i;
-        if (k == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(Cfg::kXBytes + Cfg::kLBytes + (QUANT ? 256 : 0)));
-        __syncwarp(7u << (3 * g));
-        if (k == 0)
-          tma_load_2d(st, &tm_x, &full[s], c * QB_CHUNK, m0);
-        else if (k == 1 && R > 0)
-          tma_load_2d(st + Cfg::kXBytes, &tm_l1, &full[s], c * QB_CHUNK, 0);
-        else if (k == 2 && QUANT)
-          bulk_load(st + Cfg::kXBytes + Cfg::kLBytes, inv_s + (int64_t)c * QB_CHUNK, 256, &full[s]);
+        const int c = 2 * (u_begin + i);                       // first chunk of the stage
+        const bool pair = c + 1 < nch;
+        if (xw) {
+          mbar_arrive_expect_tx(&full[s], (uint32_t)((pair ? 2 : 1) * Cfg::kXTile));
+          if (pair) tma_load_3d(st, &tm_x, &full[s], 0, m0, c);
+          else tma_load_2d(st, &tm_x1, &full[s], c * QB_CHUNK, m0);
+        } else {
+          mbar_arrive_expect_tx(&full[s], (uint32_t)((pair ? 2 : 1) * Cfg::kLTile));
+          if (pair) tma_load_3d(st + Cfg::kXBytes, &tm_l1, &full[s], 0, 0, c);
+          else tma_load_2d(st + Cfg::kXBytes, &tm_l11, &full[s], c * QB_CHUNK, 0);
+        }
+        issued = i + 1;
       }
-      __syncwarp();
-      issued = i + 1;
-    }
-    if (!ok && lane == 0) {
-      // Let the copies that were issued but not consumed land before the CTA exits.
-      int never = 0;
-      for (int i = issued > S ? issued - S : 0; i < issued; ++i)
-        mbar_wait(&full[i % S], (uint32_t)((i / S) & 1), tmo, &never, 0x203);
+      if (!ok) {
+        // Let the copies that were issued but not consumed land before the CTA exits.
+        int never = 0;
+        for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+          mbar_wait(&full[i % S], (uint32_t)((i / S) & 1), tmo, &never, 0x203);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer --
@@ -223,16 +245,22 @@ __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
         bool ok = true;
         for (int i = 0; i < my; ++i) {
           const int s = i % S;
-          if (!mbar_wait(&full[s], (uint32_t)((i / S) & 1), tmo, abort_flag, 0x211)) {
+          if (!mbar_wait_spin(&full[s], (uint32_t)((i / S) & 1), tmo, abort_flag, 0x211)) {
             ok = false;
             break;
           }
           tc_fence_after();
           uint8_t* st = smem + s * Cfg::kStageBytes;
-          const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(st));
-          const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(st + Cfg::kXBytes));
+          const int nc = 2 * (u_begin + i) + 1 < nch ? 2 : 1;     // a lone last chunk: one tile
 #pragma unroll
-          for (int j = 0; j < 4; ++j) tc_mma_bf16(tbase, adesc + 2 * j, bdesc + 2 * j, IDESC, (i | j) != 0 ? 1u : 0u);
+          for (int cc = 0; cc < Cfg::kChunks; ++cc) {
+            if (cc >= nc) break;
+            const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(st + cc * Cfg::kXTile));
+            const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(st + Cfg::kXBytes + cc * Cfg::kLTile));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc_mma_bf16(tbase, adesc + 2 * j, bdesc + 2 * j, IDESC, (i | cc | j) != 0 ? 1u : 0u);
+          }
           tc_commit(&empty[s]);
         }
         if (ok) {
@@ -250,31 +278,48 @@ __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
   } else {
     // ------------------------------------------------------------ quantizers --
     const int qi = threadIdx.x - QB_WARP_Q0 * 32;
-    const int row = qi >> 2;
-    const int g = qi & 3;
-    const int m = m0 + row;
+    const int g = qi & 3;                    // group of 16 within the chunk
+    const int cc = (qi >> 3) & 1;            // chunk within the stage
+    const int rr = 2 * (qi >> 4) + ((qi >> 2) & 1);   // rows rr and rr + 64
     const float c_x = __frcp_rn(__fmul_rn(6.0f, gs_x));
     const uint32_t KS4 = (uint32_t)(K >> 6);
     const uint32_t rcp_u32 = smem_u32(s_rcp);
     for (int i = 0; i < my; ++i) {
       const int s = i % S;
       if (!warp_wait(&full[s], (uint32_t)((i / S) & 1), tmo, abort_flag, 0x202)) break;
+      const int c = 2 * (u_begin + i) + cc;
       if constexpr (QUANT) {
-        const int c = c_begin + i;
-        const uint32_t st_u32 = smem_u32(smem + s * Cfg::kStageBytes);
-        const uint32_t inv_u32 = st_u32 + Cfg::kXBytes + Cfg::kLBytes + 64 * g;
-        const uint4 r0 = lds_v4(st_u32 + sw128(row, 2 * g));
-        const uint4 r1 = lds_v4(st_u32 + sw128(row, 2 * g + 1));
-        float4 inv[4];
+        // Every lane runs the group math and the shuffles (they take the whole warp); a lane whose chunk
+        // lies past K (the lone last chunk's partner, never loaded) only skips its stores.
+        const bool valid = c < nch;
+        {
+          const uint32_t st_u32 = smem_u32(smem + s * Cfg::kStageBytes);
+          const uint32_t x_u32 = st_u32 + cc * Cfg::kXTile;
+          // the group's 16 smoothing factors (a lane past K reads the last chunk's, never used)
+          const float4* invg =
+              reinterpret_cast<const float4*>(inv_s + (int64_t)(valid ? c : nch - 1) * QB_CHUNK + 16 * g);
+          float4 inv[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) inv[j] = lds_v4f(inv_u32 + 16 * j);
-        uint32_t w0, w1;
-        uint32_t sw = quant_group(r0, r1, inv, c_x, rcp_u32, w0, w1) << (8 * g);
-        sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
-        sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
-        if (m < M) *reinterpret_cast<uint2*>(Xq + (int64_t)m * (K >> 1) + c * 32 + 8 * g) = make_uint2(w0, w1);
-        if (g == 0 && m < Mpad)
-          *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)m, (uint32_t)c, KS4)) = sw;
+          for (int j = 0; j < 4; ++j) inv[j] = __ldg(invg + j);
+          uint4 a0 = lds_v4(x_u32 + sw128(rr, 2 * g)), a1 = lds_v4(x_u32 + sw128(rr, 2 * g + 1));
+          uint4 b0 = lds_v4(x_u32 + sw128(rr + 64, 2 * g)), b1 = lds_v4(x_u32 + sw128(rr + 64, 2 * g + 1));
+          uint32_t wa0, wa1, wb0, wb1;
+          uint32_t sa = quant_group(a0, a1, inv, c_x, rcp_u32, wa0, wa1) << (8 * g);
+          uint32_t sb = quant_group(b0, b1, inv, c_x, rcp_u32, wb0, wb1) << (8 * g);
+          sa |= __shfl_xor_sync(0xffffffffu, sa, 1);
+          sb |= __shfl_xor_sync(0xffffffffu, sb, 1);
+          sa |= __shfl_xor_sync(0xffffffffu, sa, 2);
+          sb |= __shfl_xor_sync(0xffffffffu, sb, 2);
+          const int ma = m0 + rr, mb = m0 + rr + 64;
+          if (valid && ma < M)
+            *reinterpret_cast<uint2*>(Xq + (int64_t)ma * (K >> 1) + c * 32 + 8 * g) = make_uint2(wa0, wa1);
+          if (valid && mb < M)
+            *reinterpret_cast<uint2*>(Xq + (int64_t)mb * (K >> 1) + c * 32 + 8 * g) = make_uint2(wb0, wb1);
+          if (valid && g == 0) {
+            if (ma < Mpad) *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)ma, (uint32_t)c, KS4)) = sa;
+            if (mb < Mpad) *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)mb, (uint32_t)c, KS4)) = sb;
+          }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -309,45 +354,80 @@ __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
     }
     tc_fence_before();
     if (split > 1) {
-      // Publish this CTA's partial, then take a ticket; the CTA that takes the last one reduces.
-      __threadfence();
+      // Publish this CTA's partial, then take a ticket; the CTA that takes the last one reduces.  The
+      // barrier orders every thread's partial-sum stores before thread 0's device-scope fence, which
+      // then orders them before the ticket (a release by one thread, not a fence in every thread).
       __syncthreads();
       if (threadIdx.x == 0) {
+        __threadfence();
         const unsigned old = atomicAdd(&ws_ticket[rb], 1u);
         const int last = (old % (unsigned)split) == (unsigned)split - 1u;
-        if (last) atomicExch(&ws_ticket[rb], 0u);
+        if (last) {
+          atomicExch(&ws_ticket[rb], 0u);
+          __threadfence();        // acquire: the other CTAs' partials before this CTA's reads of them
+        }
         *s_last = last;
       }
       __syncthreads();
-      __threadfence();
     } else {
       __syncthreads();
     }
     if (!*abort_flag && (split == 1 || *s_last)) {
-      for (int p = threadIdx.x; p < QB_ROWS * (R / 2); p += QB_THREADS) {
-        const int row = p / (R / 2);
-        const int col = 2 * (p % (R / 2));
-        float v0 = 0.0f, v1 = 0.0f;
+      // Four consecutive columns an item, two items a thread at once: with split > 1 every source's
+      // partial of both items is loaded before any is added (one round of loads in flight), then the
+      // sources are added in rank order.
+      constexpr int kItems = QB_ROWS * (R / 4);
+      for (int p0 = threadIdx.x; p0 < kItems; p0 += 2 * QB_THREADS) {
+        float4 v[2];
         if (split == 1) {
-          const float2 t = *reinterpret_cast<const float2*>(red + (size_t)row * R + col);
-          v0 = t.x;
-          v1 = t.y;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int p = p0 + h * QB_THREADS;
+            if (p < kItems) v[h] = *reinterpret_cast<const float4*>(red + (size_t)(p / (R / 4)) * R + 4 * (p % (R / 4)));
+          }
         } else {
-          for (int src = 0; src < split; ++src) {
-            const float2 t = __ldcg(reinterpret_cast<const float2*>(ws_part + ((size_t)src * Mpad + m0 + row) * R + col));
-            v0 += t.x;
-            v1 += t.y;
+          float4 t[2][QB_MAX_SPLIT];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int p = p0 + h * QB_THREADS;
+            if (p < kItems) {
+              const float* src0 = ws_part + ((size_t)m0 + p / (R / 4)) * R + 4 * (p % (R / 4));
+#pragma unroll
+              for (int src = 0; src < QB_MAX_SPLIT; ++src)
+                if (src < split) t[h][src] = __ldcg(reinterpret_cast<const float4*>(src0 + (size_t)src * Mpad * R));
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            v[h] = t[h][0];
+#pragma unroll
+            for (int src = 1; src < QB_MAX_SPLIT; ++src)
+              if (src < split) {
+                v[h].x += t[h][src].x;
+                v[h].y += t[h][src].y;
+                v[h].z += t[h][src].z;
+                v[h].w += t[h][src].w;
+              }
           }
         }
-        const int mm = m0 + row;
-        if (mm < M) {
-          v0 = __fmul_rn(v0, lr_scale);
-          v1 = __fmul_rn(v1, lr_scale);
-          const float h0 = __bfloat162float(__float2bfloat16_rn(v0));
-          const float h1 = __bfloat162float(__float2bfloat16_rn(v1));
-          uint16_t* d = LAs + (int64_t)mm * (2 * R) + 32 * (col >> 4) + (col & 15);
-          *reinterpret_cast<uint32_t*>(d) = pack_bf16x2(h0, h1);
-          *reinterpret_cast<uint32_t*>(d + 16) = pack_bf16x2(v0 - h0, v1 - h1);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int p = p0 + h * QB_THREADS;
+          if (p >= kItems) continue;
+          const int row = p / (R / 4);
+          const int col = 4 * (p % (R / 4));
+          const int mm = m0 + row;
+          if (mm < M) {
+            const float v4[4] = {__fmul_rn(v[h].x, lr_scale), __fmul_rn(v[h].y, lr_scale),
+                                 __fmul_rn(v[h].z, lr_scale), __fmul_rn(v[h].w, lr_scale)};
+            float hh[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) hh[e] = __bfloat162float(__float2bfloat16_rn(v4[e]));
+            uint16_t* d = LAs + (int64_t)mm * (2 * R) + 32 * (col >> 4) + (col & 15);
+            *reinterpret_cast<uint2*>(d) = make_uint2(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]));
+            *reinterpret_cast<uint2*>(d + 16) =
+                make_uint2(pack_bf16x2(v4[0] - hh[0], v4[1] - hh[1]), pack_bf16x2(v4[2] - hh[2], v4[3] - hh[3]));
+          }
         }
       }
     }

@@ -89,6 +89,21 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The rows x K bf16 matrix at `base` as a 3-D tensor {64 columns, rows, K/64 chunks} (strides 2K and
+// 128 bytes), box {64, box_rows, 2}, 128-byte swizzle: one copy brings two adjacent 64-column
+// chunks of box_rows rows and lands them as two 128-byte-swizzled tiles, one after the other.
+bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, rows, K / 64};
+  cuuint64_t strides[2] = {K * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------- checks -------
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -140,9 +155,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // {1, 2, 4, 8} that gives about one CTA per SM (the kernel runs one 576-thread CTA per SM, so a
 // larger grid would run in two waves), with at least two chunks a CTA.
 int qa_split(int64_t M, int64_t K, int sms) {
-  const int64_t rb = pad128(M) / 128, nch = K / 64;
+  const int64_t rb = pad128(M) / 128, nunits = (K / 64 + 1) / 2;   // stages of two 64-column chunks
   int split = 1;
-  while (split < QB_MAX_SPLIT && rb * 2 * split <= (int64_t)sms && nch >= 4 * split) split *= 2;
+  while (split < QB_MAX_SPLIT && rb * 2 * split <= (int64_t)sms && nunits >= 2 * split) split *= 2;
   return split;
 }
 
@@ -183,16 +198,19 @@ svdq_status launch_qa(DevInfo* d, const uint16_t* X, int64_t M, int64_t K, const
                       const uint16_t* L1fT, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
                       void* ws, cudaStream_t s) {
   using Cfg = QbCfg<R>;
-  CUtensorMap tm_x, tm_l1;
-  if (!make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64,
+  CUtensorMap tm_x, tm_l1, tm_x1, tm_l11;
+  if (!make_map_chunks(&tm_x, X, (uint64_t)K, (uint64_t)M, QB_ROWS) ||
+      !make_map_2d(&tm_x1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64,
                    QB_ROWS))
     return SVDQ_ERR_CUDA;
   if (R > 0) {
-    if (!make_map_2d(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1fT, (uint64_t)K, (uint64_t)R, (uint64_t)K * 2, 64,
+    if (!make_map_chunks(&tm_l1, L1fT, (uint64_t)K, (uint64_t)R, R > 0 ? R : 1) ||
+        !make_map_2d(&tm_l11, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1fT, (uint64_t)K, (uint64_t)R, (uint64_t)K * 2, 64,
                      R > 0 ? R : 1))
       return SVDQ_ERR_CUDA;
   } else {
     tm_l1 = tm_x;
+    tm_l11 = tm_x1;
   }
   bool& attr = d->qa_attr[QUANT ? 0 : 1][R / 16];
   if (!attr) {
@@ -207,8 +225,8 @@ svdq_status launch_qa(DevInfo* d, const uint16_t* X, int64_t M, int64_t K, const
   float* part = ws ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + qa_ticket_bytes(M)) : nullptr;
   if (R > 0 && split > 1 && !ws) return SVDQ_ERR_INVALID_ARG;
   const dim3 grid((unsigned)(Mpad / QB_ROWS * split));
-  if (launch_pdl(k_quantize_act<R, QUANT>, grid, dim3(QB_THREADS), (size_t)Cfg::kSmem, s, 1, tm_x, tm_l1,
-                 inv_s, gs_x, lr_scale, (int)M, (int)K, (int)Mpad, split, Xq, SFx, LAs, part, ticket,
+  if (launch_pdl(k_quantize_act<R, QUANT>, grid, dim3(QB_THREADS), (size_t)Cfg::kSmem, s, 1, tm_x, tm_l1, tm_x1,
+                 tm_l11, inv_s, gs_x, lr_scale, (int)M, (int)K, (int)Mpad, split, Xq, SFx, LAs, part, ticket,
                  LN_DEFAULT_TIMEOUT_NS) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return launch_status();
