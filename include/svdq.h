@@ -128,6 +128,58 @@ SVDQ_API svdq_status svdq_dequant_weight(const uint8_t* Wq, const uint8_t* SFw, 
                                 int64_t N, float* Rq, svdq_stream_t stream);
 
 /*
+ * MXFP4 form of the layer.  The pages name MXFP4 beside NVFP4 as a 4-bit
+ * format the decomposition serves (WUSH summary page, format compatibility
+ * and the MXFP4 / NVFP4 evaluations; "From SmoothQuant to SVDQuant", personal
+ * view, on group sizes) without defining it; the reading taken is the
+ * Microscaling (MX) FP4 format of its public specification:
+ *   - blocks of 32 consecutive values along K, one E8M0 scale byte e per
+ *     block standing for 2^(e - 127); no per-tensor scale;
+ *   - X = floor(log2(amax_block)) - 2 clamped to [-127, 127], e = X + 127;
+ *     code = E2M1_rne_sat(x * 2^-X) (the product is exact); a block whose
+ *     values are all zero gets e = 0 and codes 0.
+ * Codes are packed as for NVFP4.  Scales use the MMA scale order of the
+ * NVFP4 header text with KS = K/32 scales per row (4 per 32-bit word, so an
+ * atom of 512 bytes covers 128 rows x 128 values of K):
+ *   svdq_mx_sf_bytes(rows, K) = ceil(rows/128)*128*(K/32) bytes.
+ * Every MX call requires K % 128 == 0 (SVDQ_ERR_UNSUPPORTED_SHAPE otherwise).
+ */
+SVDQ_API size_t svdq_mx_sf_bytes(int64_t rows, int64_t K);
+
+/*
+ * svdq_pack_weight_mx -- MXFP4 quantization of the residual weight R
+ * (K x N float32, N contiguous) into Wq (N x K/2 codes of R^T) and SFw
+ * (svdq_mx_sf_bytes(N, K) bytes), plus the L2 layout of svdq_pack_weight
+ * (L2b r x N -> L2p N x r; both NULL when r == 0).  Two launches; no
+ * reduction over R (there is no global scale).
+ */
+SVDQ_API svdq_status svdq_pack_weight_mx(const float* R, const uint16_t* L2b, int64_t K, int64_t N, int r,
+                                         uint8_t* Wq, uint8_t* SFw, uint16_t* L2p, svdq_stream_t stream);
+
+/*
+ * svdq_quantize_act_mx -- svdq_quantize_act with the MXFP4 codec: X_hat =
+ * f32(X * inv_s) quantized in blocks of 32 to Xq (M x K/2) and SFx
+ * (svdq_mx_sf_bytes(M, K)); the fused down-projection, LAs and the workspace
+ * are exactly those of svdq_quantize_act (lr_scale is usually 1, since no
+ * global scale multiplies the product).
+ */
+SVDQ_API svdq_status svdq_quantize_act_mx(const uint16_t* X, int64_t M, int64_t K, const float* inv_s,
+                                          const uint16_t* L1fT, int r, float lr_scale, uint8_t* Xq,
+                                          uint8_t* SFx, uint16_t* LAs, void* workspace, size_t workspace_bytes,
+                                          svdq_stream_t stream);
+
+/*
+ * svdq_linear_mx -- svdq_linear on MXFP4 operands (the tcgen05 MMA of kind
+ * mxf4 with E8M0 block scales, one scale per 32 values):
+ *   Y = sum_k dec(Xq) dec(SFx) dec(Wq) dec(SFw) + LAs . L2p^T + bias,
+ * rounded once to bf16 (y_fp32 == 0) or float32.  Arguments as svdq_linear
+ * without the global scales.
+ */
+SVDQ_API svdq_status svdq_linear_mx(const uint8_t* Xq, const uint8_t* SFx, const uint8_t* Wq, const uint8_t* SFw,
+                                    const uint16_t* LAs, const uint16_t* L2p, int r, const uint16_t* bias, void* Y,
+                                    int y_fp32, int64_t M, int64_t N, int64_t K, svdq_stream_t stream);
+
+/*
  * svdq_quantize_act -- activation kernel with the fused down-projection
  * (SVDQuant review, §4.3: the down-projection is merged into the
  * quantization kernel so the activations are read once).

@@ -56,7 +56,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stdout.write(res.stdout + res.stderr)
-    for kernel in ("8k_linearE",):
+    for kernel in ("8k_linearILb0E", "8k_linearILb1E"):
         regs = entry_registers(res.stdout + res.stderr, kernel)
         if regs != LINEAR_ENTRY_REGS:
             os.remove(OUT + ".tmp")

@@ -409,6 +409,24 @@ SVDQ_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Instruction descriptor, kind::mxf4 (scale_vec::2X): A, B = E2M1 (K-major), E8M0 scales (bit 23), M x N,
+// dense K = 64; `sf_id` is the byte of the 32-bit TMEM scale column where this MMA's two scales start
+// (bits 29-30 for A, 4-5 for B).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
+         (sf_id << 29);
+}
+// D(tmem) (+)= A(smem) x B(smem)^T, E2M1 x E2M1 with E8M0 scales per 32 along K (K = 64).
+SVDQ_DEV void tc_mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                          uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor, kind::f16: A, B = bf16 (K-major), D = f32, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -443,6 +461,23 @@ SVDQ_DEV float dec_ue4m3(uint32_t b) {
   const uint16_t in = (uint16_t)(b & 0xFFu);
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// ---------------------------------------------------------------- MXFP4 -----
+// MX block scale of a block whose largest magnitude is `amax` (>= 0): the exponent
+// X = floor(log2(amax)) - 2 (2: the exponent of the largest E2M1 value, 6 = 1.5 * 2^2), clamped to
+// [-127, 127], -127 for amax = 0; returns the E8M0 byte X + 127 and sets `mul` = 2^-X (exact).
+SVDQ_DEV uint32_t mx_scale(float amax, float& mul) {
+  const uint32_t bits = __float_as_uint(amax);
+  const int e = (int)((bits >> 23) & 0xFFu);
+  int fl;
+  if (e) fl = e - 127;                                           // normal: the exponent field
+  else fl = (bits & 0x7FFFFFu) ? (31 - __clz(bits & 0x7FFFFFu)) - 149 : -129;   // subnormal / zero
+  int X = fl - 2;
+  X = X < -127 ? -127 : (X > 127 ? 127 : X);
+  const int ne = -X;                                             // 2^ne, ne in [-127, 127]
+  mul = ne >= -126 ? __uint_as_float((uint32_t)(ne + 127) << 23) : __uint_as_float(1u << 22);
+  return (uint32_t)(X + 127);
 }
 
 SVDQ_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

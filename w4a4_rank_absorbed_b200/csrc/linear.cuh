@@ -179,6 +179,10 @@ SVDQ_DEV void store_y_row(const LinearArgs& a, const uint32_t (&v)[4][32], int r
   }
 }
 
+// MX = true: the MXFP4 form (E8M0 scales per 32 along K, no global scales; K % 128 == 0).  A stage
+// of K = 256 then has two scale atoms (four scales of 32 a row each) per 128-row block, and MMA j of
+// the stage reads atom j / 2 from byte 2 (j % 2) of its TMEM columns (the scale-factor ID).
+template <bool MX>
 __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     const __grid_constant__ CUtensorMap tm_xq,   // uint8 {K/2, M},  box {128, 128}, SW128
     const __grid_constant__ CUtensorMap tm_wq,   // uint8 {K/2, N},  box {128, 128}, SW128
@@ -303,7 +307,9 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
             // Scale blocks are contiguous runs of ka 512-byte atoms, copied as they are.
             // Blocks past the end of a scale buffer (rows beyond the padded M or N) are not
             // loaded; they only feed accumulator rows or columns that are never stored.
-            const int ka = lr ? 0 : min(4, KA - 4 * kt);
+            const int KAs = MX ? (K >> 7) : KA;        // scale atoms a row block holds along K
+            const int per = MX ? 2 : 4;                // atoms per stage
+            const int ka = lr ? 0 : min(per, KAs - per * kt);
             const int has_a = mb < sfx_blocks, has_b0 = 2 * nb < sfw_blocks, has_b1 = 2 * nb + 1 < sfw_blocks;
             if (k == 0) {
               if (lr) mbar_arrive(&sf_full[stage]);        // no scales in a rank stage
@@ -313,8 +319,8 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
             __syncwarp(smask);
             if (has) {
               uint8_t* dst = k == 0 ? sSFA + stage * LN_SFA_BYTES : sSFB + stage * LN_SFB_BYTES + 2048 * (k - 1);
-              const uint8_t* src = k == 0 ? args.SFx + ((int64_t)mb * KA + 4 * kt) * 512
-                                          : args.SFw + ((int64_t)(2 * nb + k - 1) * KA + 4 * kt) * 512;
+              const uint8_t* src = k == 0 ? args.SFx + ((int64_t)mb * KAs + per * kt) * 512
+                                          : args.SFw + ((int64_t)(2 * nb + k - 1) * KAs + per * kt) * 512;
               bulk_load(dst, src, (uint32_t)(ka * 512), &sf_full[stage]);
               issued = true;
               last_parity = phase;
@@ -334,6 +340,8 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     regs_dec<LN_REGS_LOW>();
     if (lane == 0) {
       constexpr uint32_t IDESC_F4 = idesc_nvf4(LN_BM, LN_BN);
+      constexpr uint32_t IDESC_MX0 = idesc_mxf4(LN_BM, LN_BN, 0);
+      constexpr uint32_t IDESC_MX1 = idesc_mxf4(LN_BM, LN_BN, 2);
       constexpr uint32_t IDESC_BF16 = idesc_bf16(LN_BM, LN_BN);
       int stage = 0;
       uint32_t phase = 0;
@@ -355,9 +363,14 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
             const int ka = min(4, KA - 4 * kt);
             const uint32_t sfa_col = tbase + LN_SF_COL0 + LN_SF_COLS_PER_STAGE * stage;
             const uint32_t sfb_col = sfa_col + 16;
-            for (int j = 0; j < ka; ++j)
-              tc_mma_nvf4(tbase, adesc + 2 * j, bdesc + 2 * j, IDESC_F4, sfa_col + 4 * j, sfb_col + 8 * j,
-                          (kt | j) != 0 ? 1u : 0u);
+            for (int j = 0; j < ka; ++j) {
+              if constexpr (MX)
+                tc_mma_mxf4(tbase, adesc + 2 * j, bdesc + 2 * j, (j & 1) ? IDESC_MX1 : IDESC_MX0,
+                            sfa_col + 4 * (j >> 1), sfb_col + 8 * (j >> 1), (kt | j) != 0 ? 1u : 0u);
+              else
+                tc_mma_nvf4(tbase, adesc + 2 * j, bdesc + 2 * j, IDESC_F4, sfa_col + 4 * j, sfb_col + 8 * j,
+                            (kt | j) != 0 ? 1u : 0u);
+            }
           } else {
             // hi and lo of the same 16 low-rank columns meet the same 16 columns of L2p.  (With no
             // K tiles, the rank-only mode, the first rank MMA starts the accumulator.)

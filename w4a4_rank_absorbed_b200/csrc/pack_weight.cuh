@@ -109,6 +109,46 @@ __global__ void __launch_bounds__(128) k_pack_weight(const float* __restrict__ R
   *reinterpret_cast<uint32_t*>(sfw) = sfword;
 }
 
+// MXFP4 packing of R (no global scale): one thread per (column n, 128 consecutive k), four blocks of
+// 32 along K, each with its E8M0 scale (mx_scale) and codes E2M1_rne_sat(x * 2^-X) (the product is
+// exact); 64 bytes of codes and one 32-bit word of four scales.  grid: (ceil(Npad/128), K/128).
+__global__ void __launch_bounds__(128) k_pack_weight_mx(const float* __restrict__ R, int K, int N, int Npad,
+                                                        uint8_t* __restrict__ Wq, uint8_t* __restrict__ SFw) {
+  const int n = blockIdx.x * 128 + threadIdx.x;
+  const int kb = blockIdx.y;
+  if (n >= Npad) return;
+  uint8_t* sfw = SFw + sf_word_offset((uint32_t)n, (uint32_t)kb, (uint32_t)(K >> 7));
+  if (n >= N) {
+    *reinterpret_cast<uint32_t*>(sfw) = 0u;
+    return;
+  }
+  uint32_t sfword = 0u;
+  uint4* dst = reinterpret_cast<uint4*>(Wq + (int64_t)n * (K >> 1) + kb * 64);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float x[32];
+    const float* src = R + (int64_t)(kb * 128 + g * 32) * N + n;
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      x[i] = __ldg(src + (int64_t)i * N);
+      a = fmaxf(a, fabsf(x[i]));
+    }
+    float mul;
+    sfword |= mx_scale(a, mul) << (8 * g);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(x[8 * q + i], mul);
+      w[q] = a > 0.0f ? cvt_e2m1x8(v) : 0u;     // an all-zero block: codes 0
+    }
+    dst[g] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  *reinterpret_cast<uint32_t*>(sfw) = sfword;
+}
+
 // Q(R) from a packed weight: R_q[k, n] = f32(e2m1(code) * f32(dec(sb) * gs)), K x N row-major.
 // grid: (ceil(N/128), K/64); block 128; thread = (column n, 64-row slab kb), so a warp writes 32
 // consecutive columns of one row at a time.

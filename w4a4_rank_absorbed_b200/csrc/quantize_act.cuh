@@ -123,6 +123,39 @@ SVDQ_DEV uint32_t quant_group(const uint4& r0, const uint4& r1, const float4 (&i
   return sb;
 }
 
+// MXFP4: one half (16 values) of a block of 32 held by this lane and its partner (lane ^ 1): the
+// smoothing multiply, the block maximum over both halves, the E8M0 scale and the two code words.
+// Every lane of the warp must call it (it shuffles).
+SVDQ_DEV uint32_t quant_half_mx(const uint4& r0, const uint4& r1, const float4 (&inv)[4], uint32_t& w0,
+                                uint32_t& w1) {
+  const uint32_t xw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+  float2 xh[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 s4 = inv[i >> 1];
+    const float2 sp = (i & 1) ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
+    xh[i] = mul_f32x2(make_float2(bf16_lo(xw[i]), bf16_hi(xw[i])), sp);
+  }
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fmaxf(fabsf(xh[i].x), fabsf(xh[i].y)));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  float mul;
+  const uint32_t sb = mx_scale(a, mul);
+  const float2 mm = make_float2(mul, mul);
+  float q0[8], q1[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 p0 = mul_f32x2(xh[i], mm);
+    const float2 p1 = mul_f32x2(xh[4 + i], mm);
+    q0[2 * i] = p0.x; q0[2 * i + 1] = p0.y;
+    q1[2 * i] = p1.x; q1[2 * i + 1] = p1.y;
+  }
+  w0 = a > 0.0f ? cvt_e2m1x8(q0) : 0u;     // an all-zero block: codes 0
+  w1 = a > 0.0f ? cvt_e2m1x8(q1) : 0u;
+  return sb;
+}
+
 // Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
 SVDQ_DEV bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, volatile int* abort, unsigned site) {
   int ok = 1;
@@ -130,7 +163,9 @@ SVDQ_DEV bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, vol
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-template <int R, bool QUANT>
+// MX = true: the MXFP4 format (blocks of 32 with an E8M0 scale, no global scale; K % 128 == 0, so a
+// stage always holds two chunks): scale bytes follow the same MMA order with K/32 scales a row.
+template <int R, bool QUANT, bool MX = false>
 __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
     const __grid_constant__ CUtensorMap tm_x,   // bf16 {64, M, K/64} (strides 2K, 128 bytes), box {64, 128, 2}, SW128
     const __grid_constant__ CUtensorMap tm_l1,  // bf16 {64, R, K/64} (strides 2K, 128 bytes), box {64, R, 2}, SW128
@@ -303,19 +338,40 @@ __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
           for (int j = 0; j < 4; ++j) inv[j] = __ldg(invg + j);
           uint4 a0 = lds_v4(x_u32 + sw128(rr, 2 * g)), a1 = lds_v4(x_u32 + sw128(rr, 2 * g + 1));
           uint4 b0 = lds_v4(x_u32 + sw128(rr + 64, 2 * g)), b1 = lds_v4(x_u32 + sw128(rr + 64, 2 * g + 1));
-          uint32_t wa0, wa1, wb0, wb1;
-          uint32_t sa = quant_group(a0, a1, inv, c_x, rcp_u32, wa0, wa1) << (8 * g);
-          uint32_t sb = quant_group(b0, b1, inv, c_x, rcp_u32, wb0, wb1) << (8 * g);
-          sa |= __shfl_xor_sync(0xffffffffu, sa, 1);
-          sb |= __shfl_xor_sync(0xffffffffu, sb, 1);
-          sa |= __shfl_xor_sync(0xffffffffu, sa, 2);
-          sb |= __shfl_xor_sync(0xffffffffu, sb, 2);
+          uint32_t wa0, wa1, wb0, wb1, sa, sb;
+          if constexpr (MX) {
+            // the block (g / 2) of 32 spans lanes g and g ^ 1; its byte is at 2 * cc + g / 2 of the row's
+            // word for the stage (four E8M0 scales: two chunks, two blocks each)
+            // (every lane runs quant_half_mx: it shuffles with the partner lane)
+            const int sh = 8 * (2 * cc + (g >> 1));
+            const uint32_t ta = quant_half_mx(a0, a1, inv, wa0, wa1);
+            const uint32_t tb = quant_half_mx(b0, b1, inv, wb0, wb1);
+            sa = (g & 1) ? 0u : ta << sh;
+            sb = (g & 1) ? 0u : tb << sh;
+            sa |= __shfl_xor_sync(0xffffffffu, sa, 2);
+            sb |= __shfl_xor_sync(0xffffffffu, sb, 2);
+            sa |= __shfl_xor_sync(0xffffffffu, sa, 8);
+            sb |= __shfl_xor_sync(0xffffffffu, sb, 8);
+          } else {
+            sa = quant_group(a0, a1, inv, c_x, rcp_u32, wa0, wa1) << (8 * g);
+            sb = quant_group(b0, b1, inv, c_x, rcp_u32, wb0, wb1) << (8 * g);
+            sa |= __shfl_xor_sync(0xffffffffu, sa, 1);
+            sb |= __shfl_xor_sync(0xffffffffu, sb, 1);
+            sa |= __shfl_xor_sync(0xffffffffu, sa, 2);
+            sb |= __shfl_xor_sync(0xffffffffu, sb, 2);
+          }
           const int ma = m0 + rr, mb = m0 + rr + 64;
           if (valid && ma < M)
             *reinterpret_cast<uint2*>(Xq + (int64_t)ma * (K >> 1) + c * 32 + 8 * g) = make_uint2(wa0, wa1);
           if (valid && mb < M)
             *reinterpret_cast<uint2*>(Xq + (int64_t)mb * (K >> 1) + c * 32 + 8 * g) = make_uint2(wb0, wb1);
-          if (valid && g == 0) {
+          if constexpr (MX) {
+            if (valid && g == 0 && cc == 0) {
+              const uint32_t u = (uint32_t)(c >> 1), KW = (uint32_t)(K >> 7);
+              if (ma < Mpad) *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)ma, u, KW)) = sa;
+              if (mb < Mpad) *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)mb, u, KW)) = sb;
+            }
+          } else if (valid && g == 0) {
             if (ma < Mpad) *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)ma, (uint32_t)c, KS4)) = sa;
             if (mb < Mpad) *reinterpret_cast<uint32_t*>(SFx + sf_word_offset((uint32_t)mb, (uint32_t)c, KS4)) = sb;
           }

@@ -27,8 +27,8 @@ struct DevInfo {
   bool init = false;
   bool ok = false;
   int sms = 0;
-  bool linear_attr = false;
-  bool qa_attr[2][9] = {};
+  bool linear_attr[2] = {};
+  bool qa_attr[3][9] = {};      // [NVFP4 quantize, down-projection only, MXFP4 quantize][r / 16]
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -193,7 +193,7 @@ svdq_status noalloc_scratch(int dev, DevInfo* d, void** out) {
   return SVDQ_OK;
 }
 
-template <int R, bool QUANT>
+template <int R, bool QUANT, bool MX = false>
 svdq_status launch_qa(DevInfo* d, const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float gs_x,
                       const uint16_t* L1fT, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
                       void* ws, cudaStream_t s) {
@@ -212,10 +212,10 @@ svdq_status launch_qa(DevInfo* d, const uint16_t* X, int64_t M, int64_t K, const
     tm_l1 = tm_x;
     tm_l11 = tm_x1;
   }
-  bool& attr = d->qa_attr[QUANT ? 0 : 1][R / 16];
+  bool& attr = d->qa_attr[MX ? 2 : QUANT ? 0 : 1][R / 16];
   if (!attr) {
-    if (cudaFuncSetAttribute(k_quantize_act<R, QUANT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(k_quantize_act<R, QUANT, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmem) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     attr = true;
   }
@@ -225,29 +225,29 @@ svdq_status launch_qa(DevInfo* d, const uint16_t* X, int64_t M, int64_t K, const
   float* part = ws ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + qa_ticket_bytes(M)) : nullptr;
   if (R > 0 && split > 1 && !ws) return SVDQ_ERR_INVALID_ARG;
   const dim3 grid((unsigned)(Mpad / QB_ROWS * split));
-  if (launch_pdl(k_quantize_act<R, QUANT>, grid, dim3(QB_THREADS), (size_t)Cfg::kSmem, s, 1, tm_x, tm_l1, tm_x1,
+  if (launch_pdl(k_quantize_act<R, QUANT, MX>, grid, dim3(QB_THREADS), (size_t)Cfg::kSmem, s, 1, tm_x, tm_l1, tm_x1,
                  tm_l11, inv_s, gs_x, lr_scale, (int)M, (int)K, (int)Mpad, split, Xq, SFx, LAs, part, ticket,
                  LN_DEFAULT_TIMEOUT_NS) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return launch_status();
 }
 
-template <bool QUANT>
+template <bool QUANT, bool MX = false>
 svdq_status dispatch_qa(DevInfo* d, int r, const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float gs_x,
                         const uint16_t* L1fT, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs,
                         void* ws, cudaStream_t s) {
   switch (r) {
     case 0:
-      if (QUANT) return launch_qa<0, true>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+      if (QUANT) return launch_qa<0, true, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
       return SVDQ_ERR_INVALID_ARG;
-    case 16: return launch_qa<16, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
-    case 32: return launch_qa<32, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
-    case 48: return launch_qa<48, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
-    case 64: return launch_qa<64, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
-    case 80: return launch_qa<80, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
-    case 96: return launch_qa<96, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
-    case 112: return launch_qa<112, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
-    case 128: return launch_qa<128, QUANT>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 16: return launch_qa<16, QUANT, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 32: return launch_qa<32, QUANT, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 48: return launch_qa<48, QUANT, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 64: return launch_qa<64, QUANT, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 80: return launch_qa<80, QUANT, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 96: return launch_qa<96, QUANT, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 112: return launch_qa<112, QUANT, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
+    case 128: return launch_qa<128, QUANT, MX>(d, X, M, K, inv_s, gs_x, L1fT, lr_scale, Xq, SFx, LAs, ws, s);
     default: return SVDQ_ERR_UNSUPPORTED_SHAPE;
   }
 }
@@ -255,7 +255,7 @@ svdq_status dispatch_qa(DevInfo* d, int r, const uint16_t* X, int64_t M, int64_t
 svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const uint8_t* Wq, const uint8_t* SFw,
                         float gs_w, const uint16_t* LAs, const uint16_t* L2p, int r, const uint16_t* bias, void* Y,
                         int y_fp32, int64_t M, int64_t N, int64_t K, int debug, uint64_t timeout_ns,
-                        cudaStream_t s, int y_accum = 0) {
+                        cudaStream_t s, int y_accum = 0, bool mx = false) {
   // y_accum: the rank-only mode (no 4-bit operands, K = 0) that adds the up-projection into Y.
   svdq_status st = check_shape(M, N, y_accum ? 64 : K, r);
   if (st != SVDQ_OK) return st;
@@ -291,10 +291,12 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
     tm_xq = tm_las;
     tm_wq = tm_l2p;
   }
-  if (!d->linear_attr) {
-    if (cudaFuncSetAttribute(k_linear, cudaFuncAttributeMaxDynamicSharedMemorySize, LN_SMEM) != cudaSuccess)
+  if (mx && K % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!d->linear_attr[mx ? 1 : 0]) {
+    if (cudaFuncSetAttribute(mx ? k_linear<true> : k_linear<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             LN_SMEM) != cudaSuccess)
       return SVDQ_ERR_CUDA;
-    d->linear_attr = true;
+    d->linear_attr[mx ? 1 : 0] = true;
   }
   LinearArgs a;
   a.SFx = SFx;
@@ -313,8 +315,8 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   a.timeout_ns = timeout_ns ? timeout_ns : LN_DEFAULT_TIMEOUT_NS;
   const int64_t tiles = ((M + LN_BM - 1) / LN_BM) * ((N + LN_BN - 1) / LN_BN);
   const int grid = (int)(tiles < d->sms ? tiles : d->sms);
-  if (launch_pdl(k_linear, dim3(grid), dim3(LN_THREADS), (size_t)LN_SMEM, s, 1, tm_xq, tm_wq, tm_las, tm_l2p, a) !=
-      cudaSuccess)
+  if (launch_pdl(mx ? k_linear<true> : k_linear<false>, dim3(grid), dim3(LN_THREADS), (size_t)LN_SMEM, s, 1, tm_xq,
+                 tm_wq, tm_las, tm_l2p, a) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return launch_status();
 }
@@ -374,6 +376,55 @@ svdq_status svdq_pack_weight(const float* R, const uint16_t* L2b, int64_t K, int
       return SVDQ_ERR_CUDA;
   }
   return SVDQ_OK;
+}
+
+size_t svdq_mx_sf_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K < 0 || K % 128 != 0) return 0;
+  return (size_t)pad128(rows) * (size_t)(K / 32);
+}
+
+svdq_status svdq_pack_weight_mx(const float* R, const uint16_t* L2b, int64_t K, int64_t N, int r, uint8_t* Wq,
+                                uint8_t* SFw, uint16_t* L2p, svdq_stream_t stream) {
+  svdq_status st = check_shape(1, N, K, r);
+  if (st != SVDQ_OK) return st;
+  if (K % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!R || !Wq || !SFw || (r > 0 && (!L2b || !L2p))) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(R) || !aligned16(Wq) || !aligned16(SFw) || (r > 0 && (!aligned16(L2b) || !aligned16(L2p))))
+    return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t Npad = pad128(N);
+  k_pack_weight_mx<<<dim3((unsigned)(Npad / 128), (unsigned)(K / 128)), 128, 0, s>>>(R, (int)K, (int)N, (int)Npad,
+                                                                                     Wq, SFw);
+  if (r > 0) k_layout_l2<<<(unsigned)((N + 127) / 128), 128, 0, s>>>(L2b, (int)N, r, L2p);
+  return launch_status();
+}
+
+svdq_status svdq_quantize_act_mx(const uint16_t* X, int64_t M, int64_t K, const float* inv_s, const uint16_t* L1fT,
+                                 int r, float lr_scale, uint8_t* Xq, uint8_t* SFx, uint16_t* LAs, void* workspace,
+                                 size_t workspace_bytes, svdq_stream_t stream) {
+  svdq_status st = check_shape(M, 16, K, r);
+  if (st != SVDQ_OK) return st;
+  if (K % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!X || !inv_s || !Xq || !SFx || (r > 0 && (!L1fT || !LAs))) return SVDQ_ERR_INVALID_ARG;
+  if (r > 0 && (!workspace || workspace_bytes < qa_workspace_bytes(M, r))) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(inv_s) || !aligned16(Xq) || !aligned16(SFx) ||
+      (r > 0 && (!aligned16(L1fT) || !aligned16(LAs) || !aligned16(workspace))))
+    return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  return dispatch_qa<true, true>(d, r, X, M, K, inv_s, 1.0f, L1fT, lr_scale, Xq, SFx, LAs, workspace,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_linear_mx(const uint8_t* Xq, const uint8_t* SFx, const uint8_t* Wq, const uint8_t* SFw,
+                           const uint16_t* LAs, const uint16_t* L2p, int r, const uint16_t* bias, void* Y, int y_fp32,
+                           int64_t M, int64_t N, int64_t K, svdq_stream_t stream) {
+  return linear_impl(Xq, SFx, 1.0f, Wq, SFw, 1.0f, LAs, L2p, r, bias, Y, y_fp32, M, N, K, 0, 0,
+                     reinterpret_cast<cudaStream_t>(stream), 0, true);
 }
 
 svdq_status svdq_dequant_weight(const uint8_t* Wq, const uint8_t* SFw, const float* gs_w, int64_t K, int64_t N,

@@ -28,7 +28,8 @@ SVDQ_ERR_SCRATCH = 7
 
 EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_weight", "svdq_quantize_act",
             "svdq_linear", "svdq_lowrank_down", "svdq_lowrank_up", "svdq_get_device_error", "svdq_linear_debug",
-            "svdq_quantize_act_workspace_bytes", "svdq_dequant_weight", "svdq_quantize_act_noalloc")
+            "svdq_quantize_act_workspace_bytes", "svdq_dequant_weight", "svdq_quantize_act_noalloc",
+            "svdq_mx_sf_bytes", "svdq_pack_weight_mx", "svdq_quantize_act_mx", "svdq_linear_mx")
 
 
 class SVDQError(RuntimeError):
@@ -78,6 +79,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_lowrank_down.argtypes = [_P, _I64, _I64, _P, _I, _F, _P, _P, ctypes.c_size_t, _P]
     lib.svdq_lowrank_up.restype = _I
     lib.svdq_lowrank_up.argtypes = [_P, _P, _I, _F, _P, _I, _I64, _I64, _P]
+    lib.svdq_mx_sf_bytes.restype = ctypes.c_size_t
+    lib.svdq_mx_sf_bytes.argtypes = [_I64, _I64]
+    lib.svdq_pack_weight_mx.restype = _I
+    lib.svdq_pack_weight_mx.argtypes = [_P, _P, _I64, _I64, _I, _P, _P, _P, _P]
+    lib.svdq_quantize_act_mx.restype = _I
+    lib.svdq_quantize_act_mx.argtypes = [_P, _I64, _I64, _P, _P, _I, _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.svdq_linear_mx.restype = _I
+    lib.svdq_linear_mx.argtypes = [_P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I64, _I64, _I64, _P]
     lib.svdq_get_device_error.restype = _I
     lib.svdq_get_device_error.argtypes = [_P, ctypes.POINTER(_I)]
     _lib = lib
@@ -127,6 +136,38 @@ def _check(status: int, where: str):
 
 def svdq_sf_bytes(rows: int, K: int) -> int:
     return int(load_library().svdq_sf_bytes(rows, K))
+
+
+def svdq_mx_sf_bytes(rows: int, K: int) -> int:
+    return int(load_library().svdq_mx_sf_bytes(rows, K))
+
+
+def svdq_pack_weight_mx(R, L2b, K, N, r, Wq, SFw, L2p, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_pack_weight_mx(_ptr(R, torch.float32, "R"), _ptr(L2b, torch.bfloat16, "L2b"), K, N, r,
+                                 _ptr(Wq, torch.uint8, "Wq"), _ptr(SFw, torch.uint8, "SFw"),
+                                 _ptr(L2p, torch.bfloat16, "L2p"), _stream(stream))
+    _check(st, "svdq_pack_weight_mx")
+
+
+def svdq_quantize_act_mx(X, M, K, inv_s, L1fT, r, lr_scale, Xq, SFx, LAs, workspace=None, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_quantize_act_mx(_ptr(X, torch.bfloat16, "X"), M, K, _ptr(inv_s, torch.float32, "inv_s"),
+                                  _ptr(L1fT, torch.bfloat16, "L1fT"), r, float(lr_scale),
+                                  _ptr(Xq, torch.uint8, "Xq"), _ptr(SFx, torch.uint8, "SFx"),
+                                  _ptr(LAs, torch.bfloat16, "LAs"), _ptr(workspace, torch.uint8, "workspace"),
+                                  _nbytes(workspace), _stream(stream))
+    _check(st, "svdq_quantize_act_mx")
+
+
+def svdq_linear_mx(Xq, SFx, Wq, SFw, LAs, L2p, r, bias, Y, y_fp32, M, N, K, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_linear_mx(_ptr(Xq, torch.uint8, "Xq"), _ptr(SFx, torch.uint8, "SFx"),
+                            _ptr(Wq, torch.uint8, "Wq"), _ptr(SFw, torch.uint8, "SFw"),
+                            _ptr(LAs, torch.bfloat16, "LAs"), _ptr(L2p, torch.bfloat16, "L2p"), r,
+                            _ptr(bias, torch.bfloat16, "bias"), _ptr(Y, (torch.bfloat16, torch.float32), "Y"),
+                            int(y_fp32), M, N, K, _stream(stream))
+    _check(st, "svdq_linear_mx")
 
 
 def svdq_version() -> int:
