@@ -1,0 +1,157 @@
+"""The MLP pair fc1 -> GELU -> fc2 in the oracle (test infrastructure; see the package header).
+
+The pages apply the SVDQuant layer to every linear layer of a diffusion
+transformer; its MLP is fc1, a GELU, then fc2 ("SVDQuant: Absorbing Outliers
+by Low-Rank Components for 4-Bit Diffusion Models", abstract: FLUX.1;
+"From SmoothQuant to SVDQuant", section SVDQuant (W4A4)).  §4.3 of the
+SVDQuant review fuses each layer's low-rank down-projection into its
+activation quantization so that the 16-bit activations are read once; the
+fused MLP chain carries the same idea one step further: fc1's output tile
+goes through the GELU and is quantized as fc2's activations without being
+written out.  The pages define neither the activation nor the chain; the
+readings taken here:
+
+  * The activation is the tanh form of GELU,
+        GELU(y) = 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))),
+    computed in the equivalent logistic form y * sigma(2u),
+    u = sqrt(2/pi) (y + 0.044715 y^3), which has no cancellation for y < 0.
+  * Its input is fc1's output as a bf16 tensor (the value an unfused fc1
+    writes), its output is rounded once to bf16 (the value an unfused GELU
+    writes, and what fc2's quantizer reads).
+  * The arithmetic is a fixed sequence of IEEE binary32 operations, each
+    correctly rounded, so that a GPU kernel that performs the same
+    operations reproduces it bit for bit (the quantizer's decisions then
+    agree).  exp is evaluated for non-positive arguments only, by the
+    Cody-Waite range reduction (W. J. Cody and W. Waite, "Software Manual
+    for the Elementary Functions", 1980: x = n ln2 + f, ln2 split into a
+    short high part and a low part) and the Taylor polynomial of e^f to
+    degree 7 (|f| <= ln2/2, truncation below 6e-9 relative); arguments
+    below -80 return 0.
+
+  gelu_f32(y):
+      y2 = y*y;  y3 = y2*y;  w = C1*y3;  inner = y + w;  t = C2*inner      (t = 2u)
+      e = exp(-|t|);  d = 1 + e
+      sigma = 1/d if t >= 0 else e/d
+      g = y*sigma
+  with C1 = f32(0.044715), C2 = f32(2 sqrt(2/pi)).
+
+  fc1 -> fc2 chain:  Y1 (float64, the layer of oracle.linear) -> y1 = bf16(Y1)
+      -> x2 = bf16(gelu_f32(y1)) -> fc2's activation quantization and
+      low-rank down-projection (oracle.linear.quantize_act) -> fc2's layer.
+
+Pins (tests/test_oracle_mlp.py): exp against the float64 exponential over
+[-80, 0] (relative error within a few float32 ulp); gelu_f32 against the
+float64 closed form over every finite bf16 input; the closed form's
+constants against torch's float64 GELU (tanh approximation); GELU(1) against
+its decimal value; GELU(0) = 0 and GELU(-0) = -0; the odd-part identity
+GELU(y) - GELU(-y) = y; the chain against its parts on a tiny case computed
+element by element.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+from . import decompose as OD
+from . import linear as OL
+
+F32 = np.float32
+
+LOG2E = F32(1.4426950408889634)
+LN2_HI = F32(0.693145751953125)            # 16 significant bits: n * LN2_HI is exact for |n| < 256
+LN2_LO = F32(0.6931471805599453 - 0.693145751953125)
+EXP_MIN_ARG = F32(-80.0)
+C1 = F32(0.044715)
+C2 = F32(2.0 * np.sqrt(2.0 / np.pi))
+
+
+def _taylor_coeffs():
+    c = []
+    f = 1.0
+    for k in range(8):
+        if k:
+            f *= k
+        c.append(F32(1.0 / f))
+    return c
+
+
+TAYLOR = _taylor_coeffs()
+
+
+def exp_nonpos_f32(x) -> np.ndarray:
+    """e^x for float32 x <= 0 by the binary32 sequence in the module header (0 below -80)."""
+    x = np.asarray(x, dtype=F32)
+    if np.any(x > 0):
+        raise ValueError("exp_nonpos_f32 takes x <= 0")
+    with np.errstate(over="ignore", under="ignore", invalid="ignore"):
+        z = x * LOG2E
+        n = np.rint(z)
+        f = x - n * LN2_HI
+        f = f - n * LN2_LO
+        p = np.full_like(f, TAYLOR[7])
+        for k in range(6, -1, -1):
+            p = p * f + TAYLOR[k]
+        out = p * np.ldexp(F32(1.0), n.astype(np.int32)).astype(F32)
+    return np.where(x < EXP_MIN_ARG, F32(0.0), out).astype(F32)
+
+
+def gelu_f32(y) -> np.ndarray:
+    """GELU (tanh form) of float32 y by the binary32 sequence in the module header."""
+    y = np.asarray(y, dtype=F32)
+    with np.errstate(over="ignore"):            # |y| > 2^42: y^3 overflows to inf, sigma is then 0 or 1
+        y2 = y * y
+        y3 = y2 * y
+        w = C1 * y3
+        inner = y + w
+        t = C2 * inner
+    e = exp_nonpos_f32(-np.abs(t))
+    d = F32(1.0) + e
+    sigma = np.where(t >= 0, F32(1.0) / d, e / d).astype(F32)
+    return (y * sigma).astype(F32)
+
+
+def gelu_bf16(y_bf16) -> np.ndarray:
+    """bf16(gelu_f32(y)) for bf16-exact inputs (given as float64), returned as float64."""
+    y = np.asarray(y_bf16, dtype=np.float64)
+    g = gelu_f32(y.astype(F32)).astype(np.float64)
+    return OD.bf16_round(g)
+
+
+def gelu_logistic_f64(y) -> np.ndarray:
+    """The logistic form y * sigma(2u) in float64 (no cancellation for y < 0)."""
+    y = np.asarray(y, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        t = 2.0 * np.sqrt(2.0 / np.pi) * (y + 0.044715 * y ** 3)
+    e = np.exp(-np.abs(t))
+    return y * np.where(t >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def gelu_closed_form(y) -> np.ndarray:
+    """The float64 closed form 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3)))."""
+    y = np.asarray(y, dtype=np.float64)
+    return 0.5 * y * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (y + 0.044715 * y ** 3)))
+
+
+@dataclass
+class ChainFc2Input:
+    y1: np.ndarray          # M x N1: bf16(Y1), float64
+    x2: np.ndarray          # M x N1: bf16(GELU(y1)), float64 (fc2's activations)
+    qa2: OL.QuantAct        # fc2's codes, scales and X2 L1f2
+
+
+def fc2_input(Y1, inv_s2, gs_x2, L1f2: Optional[np.ndarray]) -> ChainFc2Input:
+    """What the fused fc1 epilogue produces from fc1's float64 output Y1: fc2's quantized activations."""
+    y1 = OD.bf16_round(np.asarray(Y1, dtype=np.float64))
+    x2 = gelu_bf16(y1)
+    return ChainFc2Input(y1=y1, x2=x2, qa2=OL.quantize_act(x2, inv_s2, gs_x2, L1f2))
+
+
+def mlp_reference(X, dec1, bias1, dec2, bias2):
+    """fc1 -> GELU -> fc2 with both layers as in oracle.linear.  Returns (Y2 float64, ChainFc2Input, Y1)."""
+    Y1, _, _ = OL.svdq_reference(X, dec1.inv_s, dec1.gs_x, dec1.L1f, dec1.L2b, dec1.R32, bias1)
+    c = fc2_input(Y1, dec2.inv_s, dec2.gs_x, dec2.L1f)
+    pw2 = OL.pack_weight(dec2.R32)
+    Y2 = OL.linear(c.qa2, dec2.gs_x, pw2, dec2.L2b, bias2)
+    return Y2, c, Y1
