@@ -30,8 +30,8 @@ readings taken here:
 
   gelu_f32(y):
       y2 = y*y;  y3 = y2*y;  w = C1*y3;  inner = y + w;  t = C2*inner      (t = 2u)
-      e = exp(-|t|);  d = 1 + e
-      sigma = 1/d if t >= 0 else e/d
+      e = exp(-|t|);  d = 1 + e;  q = 1/d
+      sigma = q if t >= 0 else e*q
       g = y*sigma
   with C1 = f32(0.044715), C2 = f32(2 sqrt(2/pi)).
 
@@ -108,7 +108,8 @@ def gelu_f32(y) -> np.ndarray:
         t = C2 * inner
     e = exp_nonpos_f32(-np.abs(t))
     d = F32(1.0) + e
-    sigma = np.where(t >= 0, F32(1.0) / d, e / d).astype(F32)
+    q = F32(1.0) / d
+    sigma = np.where(t >= 0, q, e * q).astype(F32)
     return (y * sigma).astype(F32)
 
 
