@@ -43,10 +43,16 @@ F32 = np.float32
 
 
 def bf16_round(a) -> np.ndarray:
-    """Round float64 to the nearest bfloat16 value, ties to even; float64 result (exact frexp/rint)."""
+    """Round float64 to the nearest bfloat16 value, ties to even; float64 result (exact frexp/rint).
+
+    bfloat16 keeps 8 significant bits down to its smallest normal 2^-126 and a fixed spacing of
+    2^-133 below it (subnormals); magnitudes that round to 2^128 or beyond become infinite."""
     a = np.asarray(a, dtype=np.float64)
-    m, e = np.frexp(a)
-    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+    _, e = np.frexp(a)                       # |a| = m 2^e, 0.5 <= m < 1
+    q = np.maximum(e - 8, -133)              # exponent of the spacing at |a|
+    r = np.ldexp(np.rint(np.ldexp(a, -q)), q)
+    with np.errstate(invalid="ignore"):
+        return np.where(np.abs(r) >= 2.0 ** 128, np.copysign(np.inf, a), r)
 
 
 def smoothing_factors(X, W, alpha: float) -> np.ndarray:

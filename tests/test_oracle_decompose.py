@@ -139,3 +139,19 @@ def test_activation_global_scale_rounds_the_product_to_float32_first():
     if rem2 * 2 > sp or (rem2 * 2 == sp and k2 % 2 == 1):
         k2 += 1
     assert got == np.float32(float(k2 * sp))
+
+
+def test_bf16_round_against_torch_conversion():
+    """bf16 rounding of the oracle against torch's float32 -> bfloat16 conversion (round to nearest even),
+    over random float32 bit patterns (normals, subnormals, values that overflow to infinity)."""
+    import torch
+    rng = np.random.default_rng(11)
+    x = rng.integers(0, 2 ** 32, 1_000_000, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    sub = np.arange(0, 2 ** 23, 13, dtype=np.uint32).view(np.float32)
+    edge = np.array([3.3895314e38, 3.4e38, -3.4e38, 0.0, -0.0, 2.0 ** -126, 2.0 ** -133, 1.5 * 2.0 ** -133],
+                    dtype=np.float32)
+    for v in (x[np.isfinite(x)], sub, -sub, edge):
+        t = torch.from_numpy(v).to(torch.bfloat16).float().numpy().astype(np.float64)
+        o = D.bf16_round(v.astype(np.float64))
+        assert np.array_equal(t, o)
+        assert np.array_equal(np.signbit(t), np.signbit(o))
