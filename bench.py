@@ -439,6 +439,55 @@ def measure_set(s, timer, dev, flush_buf):
     return out
 
 
+def mlp_chain_report(s1, s2, timer, dev):
+    """The MLP pair fc1 -> GELU -> fc2 over one batch, fused (fc1's GEMM epilogue applies GELU and
+    quantizes fc2's input: svdq_linear_gelu_quantize) against the unfused in-house pair (fc1's layer
+    writes Y1, svdq_gelu_bf16, fc2's layer reads X2), same graph protocol, rotating layer copies."""
+    import torch
+
+    from w4a4_rank_absorbed_b200 import svdq as C
+    from w4a4_rank_absorbed_b200.layer import SVDQMLP
+    M = s1["M"]
+    L1s, L2s, X1s = s1["layers"], s2["layers"], s1["Xs"]
+    n = min(len(L1s), len(L2s))
+    mlps = [SVDQMLP(L1s[i], L2s[i]) for i in range(n)]
+    Y2s = [torch.empty((M, L2s[0].N), dtype=torch.bfloat16, device=dev) for _ in range(n)]
+
+    def fused(i):
+        mlps[i % n].forward(X1s[i % n], out=Y2s[i % n], fused=True)
+
+    def unfused(i):
+        mlps[i % n].forward(X1s[i % n], out=Y2s[i % n], fused=False)
+
+    def fc1_fused_gemm(i):
+        L1, L2 = L1s[i % n], L2s[i % n]
+        L1.gemm_gelu_quantize(*L1.act_buffers(M), L2)
+
+    def gelu_only(i):
+        Y1, X2 = mlps[i % n]._mid[M]
+        C.svdq_gelu_bf16(Y1, Y1.numel(), X2)
+
+    for i in range(n):
+        unfused(i)
+        fused(i)
+    torch.cuda.synchronize()
+    d = {k: stats(timer.per_launch(f)) for k, f in (("fused", fused), ("unfused", unfused),
+                                                     ("fc1_fused_gemm", fc1_fused_gemm), ("gelu", gelu_only))}
+    K1, N1, r1 = s1["K"], s1["N"], s1["r"]
+    N2, r2 = s2["N"], s2["r"]
+    fl = layer_flops(M, K1, N1, r1) + layer_flops(M, N1, N2, r2)
+    out = {"M": M, "fc1": [K1, N1, r1], "fc2": [N1, N2, r2], "ms": d,
+           "tflops_fused": fl / (d["fused"]["median"] * 1e-3) / 1e12,
+           "tflops_unfused": fl / (d["unfused"]["median"] * 1e-3) / 1e12,
+           "speedup_fused": d["unfused"]["median"] / d["fused"]["median"],
+           "intermediate_bytes_avoided": 4.0 * M * N1,
+           "fused": "fc1 quantize, fc1 GEMM + GELU + fc2 quantize/down-projection (+ reduction), fc2 GEMM",
+           "unfused": "fc1 quantize, fc1 GEMM -> Y1 bf16, svdq_gelu_bf16, fc2 quantize, fc2 GEMM"}
+    del mlps, Y2s
+    torch.cuda.empty_cache()
+    return out
+
+
 def workload_report(s, dist_ms, hbm_peak, fp4_peak):
     M, K, N, r = s["M"], s["K"], s["N"], s["r"]
     st = {k: stats(v) for k, v in dist_ms.items()}
@@ -498,7 +547,7 @@ def run_ours(args):
     wl0 = make_workload(args.workload)
     rows = row_block(wl0.M, rank, world) if (args.strong and world > 1) else None
     del wl0
-    fc1_layer = None
+    fc1_layer = fc1_set = None
     names = [args.workload] + [w for w in (args.extra.split(",") if args.extra else []) if w and w != args.workload]
     if "fc2" in names and "fc1" not in names:
         names.insert(names.index("fc2"), "fc1")
@@ -524,9 +573,15 @@ def run_ours(args):
         if name == args.workload:
             e2e = None if args.no_e2e else e2e_leg(s, args, dev, world, dist)
             head_set = {"M": s["M"], "K": s["K"], "N": s["N"], "r": s["r"], "wl": s["wl"], "data": s["data"]}
+        if name == "fc2" and fc1_set is not None:
+            reports["mlp_chain"] = mlp_chain_report(fc1_set, s, timer, dev)
+            fc1_set = None
         if name == "fc1":
             fc1_layer = s["layers"][0]
-            s["layers"] = s["layers"][:1]
+            if "fc2" in names:
+                fc1_set = {k: s[k] for k in ("layers", "Xs", "M", "K", "N", "r")}
+            else:
+                s["layers"] = s["layers"][:1]
         del s
         torch.cuda.empty_cache()
     # Kernel 1 (offline weight packing, HBM-bound) on the headline layer: one packing of its residual R.

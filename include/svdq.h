@@ -280,6 +280,63 @@ SVDQ_API svdq_status svdq_linear(const uint8_t* Xq, const uint8_t* SFx, float gs
                         int64_t M, int64_t N, int64_t K, svdq_stream_t stream);
 
 /*
+ * svdq_linear_gelu_quantize -- the first layer of an MLP pair with the next
+ * layer's input preparation fused into its epilogue.  The pages fuse each
+ * layer's low-rank down-projection into its activation quantization so that
+ * the 16-bit activations are read from memory once (SVDQuant review, §4.3
+ * Nunchaku); between two layers of a diffusion transformer's MLP (FLUX.1,
+ * "SVDQuant: Absorbing Outliers by Low-Rank Components for 4-Bit Diffusion
+ * Models", abstract) the same reasoning removes the write and re-read of the
+ * intermediate activations altogether.  The pages define neither the
+ * activation nor this fusion; the readings taken:
+ *   - the activation is GELU in its tanh form, on the bf16-rounded output of
+ *     this layer, with its result rounded to bf16 (what an unfused pair writes
+ *     and reads): y = bf16(f32(gs_x gs_w acc + bias)), x2 = bf16(GELU(y));
+ *   - GELU(y) is the fixed binary32 sequence
+ *       t = C2 (y + C1 y^3) (products and sums each rounded: y2 = y*y, y3 = y2*y,
+ *       w = C1*y3, inner = y + w, t = C2*inner), e = exp(-|t|), q = 1/(1 + e),
+ *       GELU = y * (t >= 0 ? q : e*q),
+ *     C1 = f32(0.044715), C2 = f32(2 sqrt(2/pi)), exp by Cody-Waite reduction
+ *     and its degree-7 Taylor polynomial (0 below -80), so that its value is
+ *     reproducible bit for bit;
+ *   - the next layer then sees exactly what svdq_quantize_act would produce
+ *     from x2: codes and scales of f32(x2 * inv_s2) with global scale gs_x2,
+ *     and LAs2 = hi/lo of f32(lr_scale2 * x2 L1f2).
+ *
+ * Arguments as svdq_linear (this layer: Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p,
+ * r, bias, M, N, K; no Y), plus the next layer's constants and outputs:
+ *   inv_s2  [in]  float32, N: the next layer's smoothing factors 1/s.
+ *   gs_x2   [in]  host float > 0: the next layer's activation global scale.
+ *   L1fT2   [in]  bf16, r2 x N: the next layer's down factor (NULL if r2 == 0).
+ *   r2, lr_scale2: the next layer's rank (0, 16 or 32) and LAs pre-scale.
+ *   Xq2     [out] uint8, M x N/2;  SFx2 [out] uint8, svdq_sf_bytes(M, N).
+ *   LAs2    [out] bf16, M x 2 r2 (NULL if r2 == 0).
+ *   workspace [scratch] svdq_linear_gelu_quantize_workspace_bytes(M, N, r2)
+ *           bytes (float32 partial sums, one M x r2 slice per 256 output
+ *           columns; no initial contents needed; NULL if r2 == 0).
+ * Requires N % 64 == 0 (N is the next layer's K).  Two launches: the GEMM
+ * (its epilogue computes GELU, the next layer's codes and scales and its
+ * down-projection over each 256-column tile) and a reduction of the slices
+ * in a fixed order into LAs2.
+ */
+SVDQ_API size_t svdq_linear_gelu_quantize_workspace_bytes(int64_t M, int64_t N, int r2);
+SVDQ_API svdq_status svdq_linear_gelu_quantize(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const uint8_t* Wq,
+                                               const uint8_t* SFw, float gs_w, const uint16_t* LAs,
+                                               const uint16_t* L2p, int r, const uint16_t* bias, int64_t M,
+                                               int64_t N, int64_t K, const float* inv_s2, float gs_x2,
+                                               const uint16_t* L1fT2, int r2, float lr_scale2, uint8_t* Xq2,
+                                               uint8_t* SFx2, uint16_t* LAs2, void* workspace,
+                                               size_t workspace_bytes, svdq_stream_t stream);
+
+/*
+ * svdq_gelu_bf16 -- Y = bf16(GELU(X)) element-wise on n bf16 values, with the
+ * GELU of svdq_linear_gelu_quantize: the activation of the unfused MLP pair
+ * (svdq_linear writes the first layer's Y, this kernel applies GELU, and
+ * svdq_quantize_act reads the result).  X and Y 16-byte aligned; n >= 0.
+ */
+SVDQ_API svdq_status svdq_gelu_bf16(const uint16_t* X, int64_t n, uint16_t* Y, svdq_stream_t stream);
+
+/*
  * svdq_lowrank_down -- the low-rank down-projection as a kernel of its own: the
  * unfused form of the branch (SVDQuant review, §4.3: without fusion the branch
  * re-reads the 16-bit activations from memory, which is what the fused

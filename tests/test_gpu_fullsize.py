@@ -11,6 +11,7 @@ import torch
 
 from helpers import (GpuLayer, OC, OD, OL, bf16_dev, check_las, check_y, mismatch_report,
                      oracle_storage, require_gpu, u8_host)
+from oracle import mlp as OM
 from w4a4_rank_absorbed_b200.synth import make_workload
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -42,7 +43,7 @@ def _check_layer(wl, dec, X, what):
     rel16, mx16 = check_y(Y16.float().cpu().numpy().astype(np.float64), Y_or, bf16=True, what=what + " bf16")
     rel32, mx32 = check_y(Y32.cpu().numpy().astype(np.float64), Y_or, bf16=False, what=what + " fp32")
     print(f"{what}: bf16 rel-Fro {rel16:.3e} max/rms {mx16:.3e}; fp32 rel-Fro {rel32:.3e} max/rms {mx32:.3e}")
-    return g, Y16
+    return g, Y_or
 
 
 def test_qkv_projection():
@@ -60,10 +61,10 @@ def test_large_batch():
 def test_mlp_pair_fc1_gelu_fc2():
     wl1 = make_workload("fc1")
     dec1 = OD.decompose(wl1.X, wl1.W, wl1.r, wl1.alpha)
-    _, Y1 = _check_layer(wl1, dec1, wl1.X, "fc1")
-    # GELU (tanh form) on the harness side; fc2 is calibrated on and compared on this same bf16 tensor
-    X2 = torch.nn.functional.gelu(Y1.float(), approximate="tanh").to(torch.bfloat16)
-    X2 = X2.double().cpu().numpy()
+    _, Y1_or = _check_layer(wl1, dec1, wl1.X, "fc1")
+    # fc2's input is the oracle's GELU of the oracle's fc1 output (bf16 in, bf16 out); fc2 is
+    # calibrated on it and both sides run fc2 on it
+    X2 = OM.gelu_bf16(OD.bf16_round(Y1_or))
     wl2 = make_workload("fc2")
     wl2.X = X2
     dec2 = OD.decompose(X2, wl2.W, wl2.r, wl2.alpha)

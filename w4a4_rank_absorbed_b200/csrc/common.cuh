@@ -480,6 +480,30 @@ SVDQ_DEV uint32_t mx_scale(float amax, float& mul) {
   return (uint32_t)(X + 127);
 }
 
+// Element-wise arithmetic on float32 pairs, one packed instruction each; every element is one
+// correctly rounded operation (an explicit rounding mode: never contracted into a fused multiply-add).
+SVDQ_DEV uint64_t f2_bits(float2 a) {
+  return (uint64_t)__float_as_uint(a.x) | ((uint64_t)__float_as_uint(a.y) << 32);
+}
+SVDQ_DEV float2 bits_f2(uint64_t d) {
+  return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
+}
+SVDQ_DEV float2 mul_f32x2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+SVDQ_DEV float2 add_f32x2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+SVDQ_DEV float2 sub_f32x2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+
 SVDQ_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 SVDQ_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

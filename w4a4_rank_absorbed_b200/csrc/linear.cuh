@@ -36,6 +36,7 @@
 // scale slots of 48 columns from column 256.
 #pragma once
 #include "common.cuh"
+#include "gelu.cuh"
 
 namespace svdq {
 
@@ -64,6 +65,13 @@ constexpr int LN_OFF_SFA = LN_OFF_B + LN_STAGES * LN_B_BYTES;
 constexpr int LN_OFF_SFB = LN_OFF_SFA + LN_STAGES * LN_SFA_BYTES;
 constexpr int LN_OFF_BAR = LN_OFF_SFB + LN_STAGES * LN_SFB_BYTES;
 constexpr int LN_SMEM = LN_OFF_BAR + 256 + 1024;
+// Fused GELU + next-layer quantization epilogue: 1 KB of staging per epilogue warp (the x2 slab
+// read back by ldmatrix; a warp pair's 2 KB also carries the pair's partial-sum hand-off).
+constexpr int LN_OFF_STG = LN_OFF_BAR + 256;
+constexpr int LN_STG_BYTES = 1024;
+constexpr int LN_SMEM_GQ = LN_OFF_STG + LN_EPI_WARPS * LN_STG_BYTES + 1024;
+constexpr int LN_GQ_MAX_R = 32;
+static_assert(LN_SMEM_GQ <= 232448, "shared memory budget of the fused epilogue");
 constexpr uint64_t LN_DEFAULT_TIMEOUT_NS = 2000000000ull;
 static_assert(LN_SF_COL0 + LN_STAGES * LN_SF_COLS_PER_STAGE <= LN_TMEM_COLS, "TMEM budget");
 static_assert(LN_STAGES * LN_STREAMS <= 32 && LN_STREAMS == 3, "one lane per slot and stream");
@@ -99,7 +107,60 @@ struct LinearArgs {
   float gs;
   int debug;
   uint64_t timeout_ns;
+
+  // Fused GELU + quantization for the next layer (k_linear<..., true>): the next layer's
+  // smoothing factors (N of them), global scale and down factor (r2 x N, K-major), its codes
+  // (M x N/2), scales (MMA scale order, N/16 a row) and the partial down-projection, one
+  // Mpad x r2 float32 slice per 256-column tile of this layer's output.
+  const float* inv_s2;
+  float gs_x2;
+  const uint16_t* L1fT2;
+  int r2;
+  int Mpad;
+  uint8_t* Xq2;
+  uint8_t* SFx2;
+  float* part;
 };
+
+// Both warps of a pair (64 threads, named barrier `id`) agree that `v` holds for both.
+SVDQ_DEV bool pair_all(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 64, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return r != 0;
+}
+SVDQ_DEV void pair_sync(int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
+
+SVDQ_DEV void ldmatrix_x4(uint32_t (&a)[4], uint32_t saddr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(saddr));
+}
+
+// D += A (16 x 16 bf16, row) * B (16 x 8 bf16, col), float32 accumulate.
+SVDQ_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+SVDQ_DEV void sts_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+SVDQ_DEV void sts_v2f(uint32_t addr, float a, float b) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+SVDQ_DEV float2 lds_v2f(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
 
 // Epilogue store of one accumulator row: 128 columns from n0, y = f32(gs_x gs_w) acc + bias,
 // rounded to bf16 (or kept fp32 in test mode).  16 columns at a time: one 32-byte store of
@@ -182,7 +243,12 @@ SVDQ_DEV void store_y_row(const LinearArgs& a, const uint32_t (&v)[4][32], int r
 // MX = true: the MXFP4 form (E8M0 scales per 32 along K, no global scales; K % 128 == 0).  A stage
 // of K = 256 then has two scale atoms (four scales of 32 a row each) per 128-row block, and MMA j of
 // the stage reads atom j / 2 from byte 2 (j % 2) of its TMEM columns (the scale-factor ID).
-template <bool MX>
+// GQ = true: the epilogue does not store Y; it rounds each output to bf16, applies GELU (rounded
+// to bf16 again), and quantizes the result as the next layer's activations (NVFP4 codes and
+// scales with the next layer's smoothing factors and global scale), and multiplies it by the next
+// layer's down factor (mma.sync, bf16 in, float32 out) into one partial slice per output column
+// tile.  k_lowrank_finalize sums the slices into the next layer's LAs.
+template <bool MX, bool GQ = false>
 __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     const __grid_constant__ CUtensorMap tm_xq,   // uint8 {K/2, M},  box {128, 128}, SW128
     const __grid_constant__ CUtensorMap tm_wq,   // uint8 {K/2, N},  box {128, 128}, SW128
@@ -437,7 +503,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
         if (++stage == LN_STAGES) { stage = 0; phase ^= 1u; }
       }
     }
-  } else if (warp >= LN_EPI_WARP0) {
+  } else if (!GQ && warp >= LN_EPI_WARP0) {
     // ------------------------------------------------------------- epilogue --
     regs_inc<LN_REGS_HIGH>();
     const int ew = warp - LN_EPI_WARP0;
@@ -463,6 +529,193 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
 
       const int row = mb * LN_BM + 32 * q + lane;
       if (row < M) store_y_row(args, v, row, nb * LN_BN + h * 128, gs);
+    }
+  } else if (GQ && warp >= LN_EPI_WARP0) {
+    // ------------------------------------------- epilogue: GELU + next-layer quantization --
+    // Warp (q, h) owns rows 32 q .. +31 of the tile (lane = row) and columns h*128 .. +127.
+    regs_inc<LN_REGS_HIGH>();
+    const int ew = warp - LN_EPI_WARP0;
+    const int q = warp & 3;
+    const int h = ew >> 2;
+    const int pid = 1 + q;                           // named barrier of the warp pair (q, 0), (q, 1)
+    const float gs = args.gs;
+    const float gs2 = args.gs_x2;
+    const float c_x2 = __frcp_rn(__fmul_rn(6.0f, gs2));
+    const int r2 = args.r2;
+    const int KS4 = N >> 6;                          // scale words per row of the next layer
+    const uint32_t stg = smem_u32(smem + LN_OFF_STG + (2 * q + h) * LN_STG_BYTES);
+    const uint32_t pairbuf = smem_u32(smem + LN_OFF_STG + 2 * q * LN_STG_BYTES);
+    const int gid = lane >> 2, tig = lane & 3;
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      int mb, nb;
+      tile_coords(t, num_m, num_n, mb, nb);
+      const bool got = mbar_wait(acc_full, (uint32_t)(it & 1), tmo, abort_flag, 0x321);
+      // Both warps of the pair leave together: the named barriers below need both of them.
+      if (!pair_all(pid, got)) break;
+      tc_fence_after();
+      uint32_t v[4][32];
+      const uint32_t taddr = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * 128);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(taddr + 32 * i, v[i]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) reg_fence(v[i]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+
+      const int row = mb * LN_BM + 32 * q + lane;
+      const int n0 = nb * LN_BN + h * 128;
+      uint32_t p[64];                                // y, then x2 (bf16 pairs): p[8g + j] = columns 16g + 2j, +1
+      uint32_t cw[16];                               // codes: two words per group of 16
+      uint32_t sw[2] = {0u, 0u};                     // scale words (4 groups each)
+      // y = f32(gs acc + bias) rounded to bf16, as bf16 pairs (the accumulator registers end here,
+      // which leaves room for the GELU of several pairs at a time)
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const int n = n0 + 16 * g;
+        uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (n < N && args.bias) {                    // warp-uniform; N % 64 == 0
+          const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
+          const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(args.bias + n + 8));
+          bw[0] = b0.x; bw[1] = b0.y; bw[2] = b0.z; bw[3] = b0.w;
+          bw[4] = b1.x; bw[5] = b1.y; bw[6] = b1.z; bw[7] = b1.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float y0 = __fmaf_rn(gs, __uint_as_float(v[g >> 1][16 * (g & 1) + 2 * j]), bf16_lo(bw[j]));
+          const float y1 = __fmaf_rn(gs, __uint_as_float(v[g >> 1][16 * (g & 1) + 2 * j + 1]), bf16_hi(bw[j]));
+          p[8 * g + j] = pack_bf16x2(y0, y1);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const int n = n0 + 16 * g;
+        const bool valid = n < N;                    // warp-uniform
+        // x2 = bf16(GELU(y)), in place
+#pragma unroll
+        for (int j = 0; j < 8; ++j) p[8 * g + j] = valid ? gelu_bf16x2(p[8 * g + j]) : 0u;
+        // NVFP4 of x2 * inv_s2 with the next layer's global scale (the activation kernel's steps):
+        // one pass for the group maximum, a second (products recomputed) for the codes.
+        const float4* invp = reinterpret_cast<const float4*>(args.inv_s2 + (valid ? n : 0));
+        float2 xh[8];
+        float a = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 iv = __ldg(invp + k);
+          const uint32_t w0 = p[8 * g + 2 * k], w1 = p[8 * g + 2 * k + 1];
+          xh[2 * k] = mul_f32x2(make_float2(bf16_lo(w0), bf16_hi(w0)), make_float2(iv.x, iv.y));
+          xh[2 * k + 1] = mul_f32x2(make_float2(bf16_lo(w1), bf16_hi(w1)), make_float2(iv.z, iv.w));
+          a = fmaxf(a, fmaxf(fmaxf(fabsf(xh[2 * k].x), fabsf(xh[2 * k].y)),
+                             fmaxf(fabsf(xh[2 * k + 1].x), fabsf(xh[2 * k + 1].y))));
+        }
+        const uint32_t sb = valid ? cvt_ue4m3(__fmul_rn(a, c_x2)) : 0u;
+        const float rinv = sb ? __frcp_rn(__fmul_rn(dec_ue4m3(sb), gs2)) : 0.0f;
+        const float2 rr = make_float2(rinv, rinv);
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          float qv[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 q2 = mul_f32x2(xh[4 * hb + i], rr);
+            qv[2 * i] = q2.x;
+            qv[2 * i + 1] = q2.y;
+          }
+          cw[2 * g + hb] = sb ? cvt_e2m1x8(qv) : 0u;
+        }
+        sw[g >> 2] |= sb << (8 * (g & 3));
+      }
+      if (row < M) {
+        uint4* dst = reinterpret_cast<uint4*>(args.Xq2 + (int64_t)row * (N >> 1) + (n0 >> 1));
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (n0 + 32 * u < N) dst[u] = make_uint4(cw[4 * u], cw[4 * u + 1], cw[4 * u + 2], cw[4 * u + 3]);
+      }
+#pragma unroll
+      for (int kw = 0; kw < 2; ++kw)          // padding rows (M .. Mpad) hold zero scales
+        if (n0 + 64 * kw < N)
+          *reinterpret_cast<uint32_t*>(args.SFx2 + sf_word_offset((uint32_t)row, (uint32_t)((n0 >> 6) + kw),
+                                                                  (uint32_t)KS4)) = row < M ? sw[kw] : 0u;
+
+      if (r2 > 0) {
+        // Partial down-projection of the next layer over this warp's 128 columns:
+        // D[row][t] = sum_c x2[row][c] L1f2[n0 + c][t], 16 columns (one k step) per slab.
+        float acc2[2][LN_GQ_MAX_R / 8][4];
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+          for (int ni = 0; ni < LN_GQ_MAX_R / 8; ++ni)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc2[mi][ni][e] = 0.0f;
+#pragma unroll
+        for (int sl = 0; sl < 8; ++sl) {
+          const int kc = n0 + 16 * sl;
+          if (kc < N) {                          // warp-uniform
+            // Stage the slab (32 rows x 32 bytes; 16-byte chunk c of row L at chunk c ^ ((L >> 2) & 1),
+            // so that 8 consecutive rows of one chunk fall in 8 different bank groups).
+            __syncwarp();
+            const uint32_t sw_l = (uint32_t)((lane >> 2) & 1);
+            sts_v4(stg + lane * 32 + ((0u ^ sw_l) << 4), p[8 * sl], p[8 * sl + 1], p[8 * sl + 2], p[8 * sl + 3]);
+            sts_v4(stg + lane * 32 + ((1u ^ sw_l) << 4), p[8 * sl + 4], p[8 * sl + 5], p[8 * sl + 6], p[8 * sl + 7]);
+            __syncwarp();
+            uint32_t afr[2][4];
+#pragma unroll
+            for (int mi = 0; mi < 2; ++mi) {
+              const int j = lane >> 3;
+              const uint32_t rr = (uint32_t)(16 * mi + (j & 1) * 8 + (lane & 7));
+              const uint32_t c = (uint32_t)(j >> 1);
+              ldmatrix_x4(afr[mi], stg + rr * 32 + ((c ^ ((rr >> 2) & 1u)) << 4));
+            }
+#pragma unroll
+            for (int ni = 0; ni < LN_GQ_MAX_R / 8; ++ni) {
+              if (8 * ni < r2) {
+                const uint16_t* bp = args.L1fT2 + (int64_t)(8 * ni + gid) * N + kc + 2 * tig;
+                const uint32_t b0 = __ldg(reinterpret_cast<const unsigned int*>(bp));
+                const uint32_t b1 = __ldg(reinterpret_cast<const unsigned int*>(bp + 8));
+#pragma unroll
+                for (int mi = 0; mi < 2; ++mi) mma_bf16_16816(acc2[mi][ni], afr[mi], b0, b1);
+              }
+            }
+          }
+        }
+        // Pair hand-off, 16 columns of r2 at a time through the pair's 2 KB: warp h = 1 writes its
+        // sums, warp h = 0 adds them to its own (own + other: a fixed order) and stores the slice.
+#pragma unroll
+        for (int rh = 0; rh < LN_GQ_MAX_R / 16; ++rh) {
+          if (16 * rh < r2) {
+            pair_sync(pid);
+            if (h == 1) {
+#pragma unroll
+              for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+                for (int nj = 0; nj < 2; ++nj) {
+                  const uint32_t rr = (uint32_t)(16 * mi + gid), cc = (uint32_t)(8 * nj + 2 * tig);
+                  const float(&d)[4] = acc2[mi][2 * rh + nj];
+                  sts_v2f(pairbuf + (rr * 16 + cc) * 4, d[0], d[1]);
+                  sts_v2f(pairbuf + ((rr + 8) * 16 + cc) * 4, d[2], d[3]);
+                }
+            }
+            pair_sync(pid);
+            if (h == 0) {
+#pragma unroll
+              for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+                for (int nj = 0; nj < 2; ++nj) {
+                  const int rr = 16 * mi + gid, cc = 8 * nj + 2 * tig;
+                  const float(&d)[4] = acc2[mi][2 * rh + nj];
+                  const float2 o0 = lds_v2f(pairbuf + (uint32_t)(rr * 16 + cc) * 4);
+                  const float2 o1 = lds_v2f(pairbuf + (uint32_t)((rr + 8) * 16 + cc) * 4);
+                  const int64_t base = ((int64_t)nb * args.Mpad + mb * LN_BM + 32 * q) * r2 + 16 * rh + cc;
+                  *reinterpret_cast<float2*>(args.part + base + (int64_t)rr * r2) =
+                      make_float2(__fadd_rn(d[0], o0.x), __fadd_rn(d[1], o0.y));
+                  *reinterpret_cast<float2*>(args.part + base + (int64_t)(rr + 8) * r2) =
+                      make_float2(__fadd_rn(d[2], o1.x), __fadd_rn(d[3], o1.y));
+                }
+            }
+          }
+        }
+      }
     }
   } else {
     regs_dec<LN_REGS_LOW>();                       // warp 3: no role

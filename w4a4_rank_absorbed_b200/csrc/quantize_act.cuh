@@ -82,15 +82,6 @@ struct QbCfg {
 // Byte offset of 16-byte chunk `c16` of row `row` in a 128-byte-swizzled tile.
 SVDQ_DEV uint32_t sw128(uint32_t row, uint32_t c16) { return row * 128u + ((c16 ^ (row & 7u)) << 4); }
 
-// d = a * b element-wise on two float32 pairs (two correctly rounded products).
-SVDQ_DEV float2 mul_f32x2(float2 a, float2 b) {
-  uint64_t d;
-  const uint64_t x = (uint64_t)__float_as_uint(a.x) | ((uint64_t)__float_as_uint(a.y) << 32);
-  const uint64_t y = (uint64_t)__float_as_uint(b.x) | ((uint64_t)__float_as_uint(b.y) << 32);
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(y));
-  return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
-}
-
 // One group of 16 values of X (two 16-byte smem chunks) times 16 smoothing factors:
 // returns the UE4M3 scale and the two 32-bit code words.
 SVDQ_DEV uint32_t quant_group(const uint4& r0, const uint4& r1, const float4 (&inv)[4], float c_x,

@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -27,7 +29,7 @@ struct DevInfo {
   bool init = false;
   bool ok = false;
   int sms = 0;
-  bool linear_attr[2] = {};
+  bool linear_attr[3] = {};     // [NVFP4, MXFP4, NVFP4 with the GELU + next-layer quantization epilogue]
   bool qa_attr[3][9] = {};      // [NVFP4 quantize, down-projection only, MXFP4 quantize][r / 16]
 };
 DevInfo g_dev[kMaxDevices];
@@ -252,20 +254,48 @@ svdq_status dispatch_qa(DevInfo* d, int r, const uint16_t* X, int64_t M, int64_t
   }
 }
 
+// The next layer's quantization done in the GEMM epilogue (svdq_linear_gelu_quantize).
+struct GqArgs {
+  const float* inv_s2;
+  float gs_x2;
+  const uint16_t* L1fT2;
+  int r2;
+  float lr_scale2;
+  uint8_t* Xq2;
+  uint8_t* SFx2;
+  uint16_t* LAs2;
+  float* part;
+};
+
+size_t gq_workspace_bytes(int64_t M, int64_t N, int r2) {
+  if (r2 <= 0) return 0;
+  return (size_t)((N + LN_BN - 1) / LN_BN) * (size_t)pad128(M) * (size_t)r2 * sizeof(float);
+}
+
 svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const uint8_t* Wq, const uint8_t* SFw,
                         float gs_w, const uint16_t* LAs, const uint16_t* L2p, int r, const uint16_t* bias, void* Y,
                         int y_fp32, int64_t M, int64_t N, int64_t K, int debug, uint64_t timeout_ns,
-                        cudaStream_t s, int y_accum = 0, bool mx = false) {
+                        cudaStream_t s, int y_accum = 0, bool mx = false, const GqArgs* gq = nullptr) {
   // y_accum: the rank-only mode (no 4-bit operands, K = 0) that adds the up-projection into Y.
+  // gq: no Y; the epilogue writes the next layer's quantized activations instead.
   svdq_status st = check_shape(M, N, y_accum ? 64 : K, r);
   if (st != SVDQ_OK) return st;
   if (y_accum ? (r == 0 || !LAs || !L2p || !Y || bias)
-              : (!Xq || !SFx || !Wq || !SFw || !Y || (r > 0 && (!LAs || !L2p))))
+              : (!Xq || !SFx || !Wq || !SFw || (!gq && !Y) || (r > 0 && (!LAs || !L2p))))
     return SVDQ_ERR_INVALID_ARG;
   if (y_fp32 != 0 && y_fp32 != 1) return SVDQ_ERR_INVALID_ARG;
-  if ((!y_accum && (!aligned16(Xq) || !aligned16(SFx) || !aligned16(Wq) || !aligned16(SFw))) || !aligned16(Y) ||
-      (bias && !aligned16(bias)) || (r > 0 && (!aligned16(LAs) || !aligned16(L2p))))
+  if ((!y_accum && (!aligned16(Xq) || !aligned16(SFx) || !aligned16(Wq) || !aligned16(SFw))) ||
+      (!gq && !aligned16(Y)) || (bias && !aligned16(bias)) || (r > 0 && (!aligned16(LAs) || !aligned16(L2p))))
     return SVDQ_ERR_MISALIGNED;
+  if (gq) {
+    if (N % 64 != 0 || (gq->r2 != 0 && gq->r2 != 16 && gq->r2 != 32)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    if (!gq->inv_s2 || !gq->Xq2 || !gq->SFx2 || !(gq->gs_x2 > 0.0f) || !std::isfinite(gq->gs_x2) ||
+        (gq->r2 > 0 && (!gq->L1fT2 || !gq->LAs2 || !gq->part)))
+      return SVDQ_ERR_INVALID_ARG;
+    if (!aligned16(gq->inv_s2) || !aligned16(gq->Xq2) || !aligned16(gq->SFx2) ||
+        (gq->r2 > 0 && (!aligned16(gq->L1fT2) || !aligned16(gq->LAs2) || !aligned16(gq->part))))
+      return SVDQ_ERR_MISALIGNED;
+  }
   int dev;
   DevInfo* d;
   if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
@@ -292,11 +322,13 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
     tm_wq = tm_l2p;
   }
   if (mx && K % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-  if (!d->linear_attr[mx ? 1 : 0]) {
-    if (cudaFuncSetAttribute(mx ? k_linear<true> : k_linear<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             LN_SMEM) != cudaSuccess)
+  const int variant = gq ? 2 : mx ? 1 : 0;
+  auto kernel = gq ? k_linear<false, true> : mx ? k_linear<true, false> : k_linear<false, false>;
+  const int smem_bytes = gq ? LN_SMEM_GQ : LN_SMEM;
+  if (!d->linear_attr[variant]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
       return SVDQ_ERR_CUDA;
-    d->linear_attr[mx ? 1 : 0] = true;
+    d->linear_attr[variant] = true;
   }
   LinearArgs a;
   a.SFx = SFx;
@@ -313,11 +345,26 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   a.gs = gs_x * gs_w;
   a.debug = debug;
   a.timeout_ns = timeout_ns ? timeout_ns : LN_DEFAULT_TIMEOUT_NS;
+  a.inv_s2 = gq ? gq->inv_s2 : nullptr;
+  a.gs_x2 = gq ? gq->gs_x2 : 1.0f;
+  a.L1fT2 = gq ? gq->L1fT2 : nullptr;
+  a.r2 = gq ? gq->r2 : 0;
+  a.Mpad = (int)pad128(M);
+  a.Xq2 = gq ? gq->Xq2 : nullptr;
+  a.SFx2 = gq ? gq->SFx2 : nullptr;
+  a.part = gq ? gq->part : nullptr;
   const int64_t tiles = ((M + LN_BM - 1) / LN_BM) * ((N + LN_BN - 1) / LN_BN);
   const int grid = (int)(tiles < d->sms ? tiles : d->sms);
-  if (launch_pdl(mx ? k_linear<true> : k_linear<false>, dim3(grid), dim3(LN_THREADS), (size_t)LN_SMEM, s, 1, tm_xq,
-                 tm_wq, tm_las, tm_l2p, a) != cudaSuccess)
+  if (launch_pdl(kernel, dim3(grid), dim3(LN_THREADS), (size_t)smem_bytes, s, 1, tm_xq, tm_wq, tm_las, tm_l2p, a) !=
+      cudaSuccess)
     return SVDQ_ERR_CUDA;
+  if (gq && gq->r2 > 0) {
+    const int items = (int)M * (gq->r2 / 4);
+    if (launch_pdl(k_lowrank_finalize, dim3((items + 255) / 256), dim3(256), 0, s, 1, (const float*)gq->part,
+                   (int)((N + LN_BN - 1) / LN_BN), (int)M, (int)pad128(M), gq->r2, gq->lr_scale2, gq->LAs2) !=
+        cudaSuccess)
+      return SVDQ_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -425,6 +472,52 @@ svdq_status svdq_linear_mx(const uint8_t* Xq, const uint8_t* SFx, const uint8_t*
                            int64_t M, int64_t N, int64_t K, svdq_stream_t stream) {
   return linear_impl(Xq, SFx, 1.0f, Wq, SFw, 1.0f, LAs, L2p, r, bias, Y, y_fp32, M, N, K, 0, 0,
                      reinterpret_cast<cudaStream_t>(stream), 0, true);
+}
+
+size_t svdq_linear_gelu_quantize_workspace_bytes(int64_t M, int64_t N, int r2) {
+  if (M < 1 || N < 1 || r2 < 0) return 0;
+  return gq_workspace_bytes(M, N, r2);
+}
+
+svdq_status svdq_linear_gelu_quantize(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const uint8_t* Wq,
+                                      const uint8_t* SFw, float gs_w, const uint16_t* LAs, const uint16_t* L2p, int r,
+                                      const uint16_t* bias, int64_t M, int64_t N, int64_t K, const float* inv_s2,
+                                      float gs_x2, const uint16_t* L1fT2, int r2, float lr_scale2, uint8_t* Xq2,
+                                      uint8_t* SFx2, uint16_t* LAs2, void* workspace, size_t workspace_bytes,
+                                      svdq_stream_t stream) {
+  svdq_status st = check_shape(M, N, K, r);
+  if (st != SVDQ_OK) return st;
+  if (N % 64 != 0 || (r2 != 0 && r2 != 16 && r2 != 32)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (r2 > 0 && workspace_bytes < gq_workspace_bytes(M, N, r2)) return SVDQ_ERR_INVALID_ARG;
+  GqArgs g;
+  g.inv_s2 = inv_s2;
+  g.gs_x2 = gs_x2;
+  g.L1fT2 = L1fT2;
+  g.r2 = r2;
+  g.lr_scale2 = lr_scale2;
+  g.Xq2 = Xq2;
+  g.SFx2 = SFx2;
+  g.LAs2 = LAs2;
+  g.part = static_cast<float*>(workspace);
+  return linear_impl(Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p, r, bias, nullptr, 0, M, N, K, 0, 0,
+                     reinterpret_cast<cudaStream_t>(stream), 0, false, &g);
+}
+
+svdq_status svdq_gelu_bf16(const uint16_t* X, int64_t n, uint16_t* Y, svdq_stream_t stream) {
+  if (n < 0 || (n > 0 && (!X || !Y))) return SVDQ_ERR_INVALID_ARG;
+  if (n == 0) return SVDQ_OK;
+  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  svdq_status st;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  const int64_t nv = (n + 7) / 8;
+  const int64_t cap = (int64_t)d->sms * 8;
+  const int blocks = (int)std::min<int64_t>((nv + 255) / 256, cap);
+  if (launch_pdl(k_gelu_bf16, dim3(blocks), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), 1, X, n, Y) !=
+      cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  return launch_status();
 }
 
 svdq_status svdq_dequant_weight(const uint8_t* Wq, const uint8_t* SFw, const float* gs_w, int64_t K, int64_t N,

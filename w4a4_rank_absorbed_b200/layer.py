@@ -100,6 +100,24 @@ class SVDQLinear:
                            Y, 1 if Y.dtype == torch.float32 else 0, M, self.N, self.K, stream)
         return Y
 
+    def gemm_gelu_quantize(self, Xq, SFx, LAs, nxt: "SVDQLinear", stream=None):
+        """This layer's GEMM with GELU and `nxt`'s activation quantization in its epilogue (no Y is
+        written); returns nxt's quantized activations (Xq2, SFx2, LAs2), ready for nxt.gemm."""
+        for t, name in ((Xq, "Xq"), (SFx, "SFx"), (LAs, "LAs")):
+            check_device(t, self.device, name)
+        if nxt.device != self.device or nxt.K != self.N:
+            raise ValueError("the next layer must be on the same device and take this layer's N as its K")
+        M = Xq.shape[0]
+        Xq2, SFx2, LAs2 = nxt.act_buffers(M)
+        key = ("gq", M, nxt.r)
+        if key not in self._act:
+            self._act[key] = _C.new_gelu_quantize_workspace(M, self.N, nxt.r, self.device)
+        with torch.cuda.device(self.device):
+            _C.svdq_linear_gelu_quantize(Xq, SFx, self.gs_x, self.Wq, self.SFw, self.gs_w, LAs, self.L2p, self.r,
+                                         self.bias, M, self.N, self.K, nxt.inv_s, nxt.gs_x, nxt.L1fT, nxt.r,
+                                         nxt.lr_scale, Xq2, SFx2, LAs2, self._act[key], stream)
+        return Xq2, SFx2, LAs2
+
     def forward(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, y_fp32: bool = False,
                 stream=None) -> torch.Tensor:
         """Y = layer(X); X bf16 [M, K] on the device; returns bf16 (or fp32) [M, N]."""
@@ -160,3 +178,40 @@ class SVDQLinear:
                 done_out[b].record(s_out)
         for st in (s_in, s_cmp, s_out):
             cur.wait_stream(st)
+
+
+class SVDQMLP:
+    """Two SVDQuant layers with GELU (tanh form) between them, fc2(GELU(fc1(X))).
+
+    fused=True (the default): three launches of the library per call plus the small reduction of
+    fc2's down-projection: fc1's activation kernel, fc1's GEMM whose epilogue applies GELU and
+    quantizes the result as fc2's activations (svdq_linear_gelu_quantize), fc2's GEMM.  fused=False
+    runs the unfused pair: fc1's layer, svdq_gelu_bf16, fc2's layer (fc1's output makes a round trip
+    through memory as bf16)."""
+
+    def __init__(self, fc1: SVDQLinear, fc2: SVDQLinear):
+        if fc2.K != fc1.N or fc2.device != fc1.device:
+            raise ValueError("fc2 must take fc1's output on the same device")
+        self.fc1, self.fc2 = fc1, fc2
+        self._mid: Dict[int, torch.Tensor] = {}
+
+    def forward(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, fused: bool = True,
+                stream=None) -> torch.Tensor:
+        fc1, fc2 = self.fc1, self.fc2
+        M = X.shape[0]
+        if out is None:
+            out = torch.empty((M, fc2.N), dtype=torch.bfloat16, device=fc1.device)
+        check_device(out, fc1.device, "out")
+        if fused:
+            Xq, SFx, LAs = fc1.quantize(X, stream)
+            return fc2.gemm(*fc1.gemm_gelu_quantize(Xq, SFx, LAs, fc2, stream), out, stream)
+        if M not in self._mid:
+            self._mid[M] = (torch.empty((M, fc1.N), dtype=torch.bfloat16, device=fc1.device),
+                            torch.empty((M, fc1.N), dtype=torch.bfloat16, device=fc1.device))
+        Y1, X2 = self._mid[M]
+        fc1.forward(X, out=Y1, stream=stream)
+        with torch.cuda.device(fc1.device):
+            _C.svdq_gelu_bf16(Y1, Y1.numel(), X2, stream)
+        return fc2.forward(X2, out=out, stream=stream)
+
+    __call__ = forward

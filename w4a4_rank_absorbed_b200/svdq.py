@@ -29,7 +29,8 @@ SVDQ_ERR_SCRATCH = 7
 EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_weight", "svdq_quantize_act",
             "svdq_linear", "svdq_lowrank_down", "svdq_lowrank_up", "svdq_get_device_error", "svdq_linear_debug",
             "svdq_quantize_act_workspace_bytes", "svdq_dequant_weight", "svdq_quantize_act_noalloc",
-            "svdq_mx_sf_bytes", "svdq_pack_weight_mx", "svdq_quantize_act_mx", "svdq_linear_mx")
+            "svdq_mx_sf_bytes", "svdq_pack_weight_mx", "svdq_quantize_act_mx", "svdq_linear_mx",
+            "svdq_linear_gelu_quantize", "svdq_linear_gelu_quantize_workspace_bytes", "svdq_gelu_bf16")
 
 
 class SVDQError(RuntimeError):
@@ -87,6 +88,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_quantize_act_mx.argtypes = [_P, _I64, _I64, _P, _P, _I, _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
     lib.svdq_linear_mx.restype = _I
     lib.svdq_linear_mx.argtypes = [_P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I64, _I64, _I64, _P]
+    lib.svdq_linear_gelu_quantize_workspace_bytes.restype = ctypes.c_size_t
+    lib.svdq_linear_gelu_quantize_workspace_bytes.argtypes = [_I64, _I64, _I]
+    lib.svdq_linear_gelu_quantize.restype = _I
+    lib.svdq_linear_gelu_quantize.argtypes = [_P, _P, _F, _P, _P, _F, _P, _P, _I, _P, _I64, _I64, _I64, _P, _F, _P, _I,
+                                              _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.svdq_gelu_bf16.restype = _I
+    lib.svdq_gelu_bf16.argtypes = [_P, _I64, _P, _P]
     lib.svdq_get_device_error.restype = _I
     lib.svdq_get_device_error.argtypes = [_P, ctypes.POINTER(_I)]
     _lib = lib
@@ -168,6 +176,35 @@ def svdq_linear_mx(Xq, SFx, Wq, SFw, LAs, L2p, r, bias, Y, y_fp32, M, N, K, stre
                             _ptr(bias, torch.bfloat16, "bias"), _ptr(Y, (torch.bfloat16, torch.float32), "Y"),
                             int(y_fp32), M, N, K, _stream(stream))
     _check(st, "svdq_linear_mx")
+
+
+def svdq_linear_gelu_quantize_workspace_bytes(M: int, N: int, r2: int) -> int:
+    return int(load_library().svdq_linear_gelu_quantize_workspace_bytes(M, N, r2))
+
+
+def new_gelu_quantize_workspace(M: int, N: int, r2: int, device=None) -> Optional[torch.Tensor]:
+    """Scratch for svdq_linear_gelu_quantize (None when none is needed); its contents need no initial value."""
+    n = svdq_linear_gelu_quantize_workspace_bytes(M, N, r2)
+    return torch.empty(n, dtype=torch.uint8, device=device if device is not None else "cuda") if n else None
+
+
+def svdq_linear_gelu_quantize(Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p, r, bias, M, N, K, inv_s2, gs_x2, L1fT2, r2,
+                              lr_scale2, Xq2, SFx2, LAs2, workspace=None, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_linear_gelu_quantize(
+        _ptr(Xq, torch.uint8, "Xq"), _ptr(SFx, torch.uint8, "SFx"), float(gs_x), _ptr(Wq, torch.uint8, "Wq"),
+        _ptr(SFw, torch.uint8, "SFw"), float(gs_w), _ptr(LAs, torch.bfloat16, "LAs"), _ptr(L2p, torch.bfloat16, "L2p"),
+        r, _ptr(bias, torch.bfloat16, "bias"), M, N, K, _ptr(inv_s2, torch.float32, "inv_s2"), float(gs_x2),
+        _ptr(L1fT2, torch.bfloat16, "L1fT2"), r2, float(lr_scale2), _ptr(Xq2, torch.uint8, "Xq2"),
+        _ptr(SFx2, torch.uint8, "SFx2"), _ptr(LAs2, torch.bfloat16, "LAs2"), _ptr(workspace, torch.uint8, "workspace"),
+        _nbytes(workspace), _stream(stream))
+    _check(st, "svdq_linear_gelu_quantize")
+
+
+def svdq_gelu_bf16(X, n, Y, stream=None) -> None:
+    lib = load_library()
+    st = lib.svdq_gelu_bf16(_ptr(X, torch.bfloat16, "X"), n, _ptr(Y, torch.bfloat16, "Y"), _stream(stream))
+    _check(st, "svdq_gelu_bf16")
 
 
 def svdq_version() -> int:
