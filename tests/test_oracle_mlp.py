@@ -27,6 +27,15 @@ def test_exp_against_float64_exponential():
         OM.exp_nonpos_f32(np.float32(1.0))
 
 
+def test_reciprocal_on_one_to_two():
+    d = np.linspace(1.0, 2.0, 1000001).astype(np.float32)
+    q = OM.recip_1_2(d).astype(np.float64)
+    exact = 1.0 / d.astype(np.float64)
+    assert np.max(np.abs(q - exact) / exact) <= 1.5 * 2.0 ** -24
+    assert OM.recip_1_2(np.float32(1.0)) == 1.0 and OM.recip_1_2(np.float32(2.0)) == 0.5
+    assert float(OM.R0A) == pytest.approx(24.0 / 17.0, rel=1e-7) and float(OM.R0B) == pytest.approx(8.0 / 17.0, rel=1e-7)
+
+
 def test_taylor_coefficients_are_reciprocal_factorials():
     for k, c in enumerate(OM.TAYLOR):
         assert c == np.float32(1.0 / math.factorial(k))
