@@ -19,26 +19,29 @@ readings taken here:
     writes), its output is rounded once to bf16 (the value an unfused GELU
     writes, and what fc2's quantizer reads).
   * The arithmetic is a fixed sequence of IEEE binary32 operations, each
-    correctly rounded, so that a GPU kernel that performs the same
-    operations reproduces it bit for bit (the quantizer's decisions then
-    agree).  exp is evaluated for non-positive arguments only, by the
-    Cody-Waite range reduction (W. J. Cody and W. Waite, "Software Manual
-    for the Elementary Functions", 1980: x = n ln2 + f, ln2 split into a
-    short high part and a low part) and the Taylor polynomial of e^f to
-    degree 7 (|f| <= ln2/2, truncation below 6e-9 relative); arguments
-    below -80 return 0.
+    correctly rounded (a fused multiply-add fma(a, b, c) = a*b + c rounded
+    once), so that a GPU kernel that performs the same operations
+    reproduces it bit for bit (the quantizer's decisions then agree).  exp
+    is evaluated for arguments in [-80, 0] by the Cody-Waite range
+    reduction (W. J. Cody and W. Waite, "Software Manual for the Elementary
+    Functions", 1980: x = n ln2 + f, ln2 split into a short high part and a
+    low part) and the Taylor polynomial of e^f to degree 6 (|f| <= ln2/2:
+    truncation below 1.2e-7 relative); 1/(1 + e) by Newton's iteration.
 
   gelu_f32(y):
-      y2 = y*y;  y3 = y2*y;  w = C1*y3;  inner = y + w;  t = C2*inner      (t = 2u)
-      e = exp(-|t|);  d = 1 + e  (in [1, 2])
-      q = 1/d by Newton's iteration from the linear seed q0 = R0A - R0B*d
-          (R0A = f32(24/17), R0B = f32(8/17): relative error at most 1/17 on
-          [1, 2]), three steps q <- q + q*(1 - d*q), each a multiplication,
-          a subtraction, a multiplication and an addition (within 1.5 ulp of
-          1/d; no division, no branch)
+      y2 = y*y;  h = fma(C3, y2, C2);  t = y*h                (t = 2u)
+      x = -|t|
+      a = fma(x, LOG2E, 1.5 2^23);  nf = a - 1.5 2^23        (nf = rint(x log2 e))
+      f = fma(-nf, LN2_HI, x);  f = fma(-nf, LN2_LO, f)
+      p = 1/6!;  p = fma(p, f, 1/k!) for k = 5 .. 0
+      e = p * 2^nf  if x >= -80, else 0                      (e = exp(x))
+      d = 1 + e                                              (in [1, 2])
+      q = fma(-R0B, d, R0A), then three times: r = fma(-d, q, 1); q = fma(q, r, q)
+          (Newton's iteration for 1/d from a linear seed of relative error
+          at most 1/17: R0A = f32(24/17), R0B = f32(8/17))
       sigma = q if t >= 0 else e*q
       g = y*sigma
-  with C1 = f32(0.044715), C2 = f32(2 sqrt(2/pi)).
+  with C2 = f32(2 sqrt(2/pi)), C3 = f32(C2 * 0.044715).
 
   fc1 -> fc2 chain:  Y1 (float64, the layer of oracle.linear) -> y1 = bf16(Y1)
       -> x2 = bf16(gelu_f32(y1)) -> fc2's activation quantization and
@@ -68,11 +71,13 @@ F32 = np.float32
 LOG2E = F32(1.4426950408889634)
 LN2_HI = F32(0.693145751953125)            # 16 significant bits: n * LN2_HI is exact for |n| < 256
 LN2_LO = F32(0.6931471805599453 - 0.693145751953125)
+MAGIC = F32(12582912.0)                    # 1.5 * 2^23: adding it rounds to an integer
 EXP_MIN_ARG = F32(-80.0)
 R0A = F32(24.0 / 17.0)
 R0B = F32(8.0 / 17.0)
-C1 = F32(0.044715)
 C2 = F32(2.0 * np.sqrt(2.0 / np.pi))
+C3 = F32(2.0 * np.sqrt(2.0 / np.pi) * 0.044715)
+TAYLOR_DEGREE = 6
 
 
 def _taylor_coeffs():
@@ -88,45 +93,64 @@ def _taylor_coeffs():
 TAYLOR = _taylor_coeffs()
 
 
-def exp_nonpos_f32(x) -> np.ndarray:
-    """e^x for float32 x <= 0 by the binary32 sequence in the module header (0 below -80)."""
+def fma32(a, b, c) -> np.ndarray:
+    """a*b + c rounded once to binary32 (round to nearest even), for binary32 a, b, c.
+
+    a*b is exact in float64 (48 significant bits); s = a*b + c is rounded to float64 with its
+    exact error err (TwoSum).  Rounding s to binary32 gives the right answer except when s sits
+    exactly on a binary32 midpoint (binary32 midpoints are float64 numbers, so rounding to float64
+    can land on one but not cross it); there the exact value lies on err's side."""
+    A = np.asarray(a, dtype=F32).astype(np.float64)
+    B = np.asarray(b, dtype=F32).astype(np.float64)
+    C = np.asarray(c, dtype=F32).astype(np.float64)
+    p = A * B
+    with np.errstate(over="ignore", invalid="ignore"):
+        s = p + C
+        bb = s - p
+        err = (p - (s - bb)) + (C - bb)
+        r = s.astype(F32)
+        other = np.where(r.astype(np.float64) < s, np.nextafter(r, F32(np.inf)), np.nextafter(r, F32(-np.inf)))
+        mid = (s == (r.astype(np.float64) + other.astype(np.float64)) / 2.0) & np.isfinite(s)
+        fix = mid & (err != 0)
+        toward_up = err > 0
+        pick = np.where(toward_up, np.maximum(r, other), np.minimum(r, other))
+    return np.where(fix, pick, r).astype(F32)
+
+
+def exp_m80_0_f32(x) -> np.ndarray:
+    """e^x for float32 x in [-80, 0] by the binary32 sequence in the module header."""
     x = np.asarray(x, dtype=F32)
-    if np.any(x > 0):
-        raise ValueError("exp_nonpos_f32 takes x <= 0")
-    with np.errstate(over="ignore", under="ignore", invalid="ignore"):
-        z = x * LOG2E
-        n = np.rint(z)
-        f = x - n * LN2_HI
-        f = f - n * LN2_LO
-        p = np.full_like(f, TAYLOR[7])
-        for k in range(6, -1, -1):
-            p = p * f + TAYLOR[k]
-        out = p * np.ldexp(F32(1.0), n.astype(np.int32)).astype(F32)
-    return np.where(x < EXP_MIN_ARG, F32(0.0), out).astype(F32)
+    if np.any(x > 0) or np.any(x < EXP_MIN_ARG):
+        raise ValueError("exp_m80_0_f32 takes -80 <= x <= 0")
+    a = fma32(x, LOG2E, MAGIC)
+    nf = a - MAGIC
+    f = fma32(-nf, LN2_HI, x)
+    f = fma32(-nf, LN2_LO, f)
+    p = np.full_like(f, TAYLOR[TAYLOR_DEGREE])
+    for k in range(TAYLOR_DEGREE - 1, -1, -1):
+        p = fma32(p, f, TAYLOR[k])
+    return (p * np.ldexp(F32(1.0), nf.astype(np.int32)).astype(F32)).astype(F32)
 
 
 def recip_1_2(d) -> np.ndarray:
     """1/d for float32 d in [1, 2]: Newton's iteration from a linear seed, the sequence in the module header."""
     d = np.asarray(d, dtype=F32)
-    q = R0A - R0B * d
+    q = fma32(-R0B, d, R0A)
     for _ in range(3):
-        u = d * q
-        v = F32(1.0) - u
-        w = q * v
-        q = q + w
-    return q.astype(F32)
+        r = fma32(-d, q, F32(1.0))
+        q = fma32(q, r, q)
+    return q
 
 
 def gelu_f32(y) -> np.ndarray:
     """GELU (tanh form) of float32 y by the binary32 sequence in the module header."""
     y = np.asarray(y, dtype=F32)
-    with np.errstate(over="ignore"):            # |y| > 2^42: y^3 overflows to inf, sigma is then 0 or 1
+    with np.errstate(over="ignore", invalid="ignore"):   # |y| > 2^64: y^2 overflows, t = +-inf
         y2 = y * y
-        y3 = y2 * y
-        w = C1 * y3
-        inner = y + w
-        t = C2 * inner
-    e = exp_nonpos_f32(-np.abs(t))
+        h = fma32(C3, y2, C2)
+        t = y * h
+    x = (-np.abs(t)).astype(F32)
+    e = np.where(x < EXP_MIN_ARG, F32(0.0), exp_m80_0_f32(np.maximum(x, EXP_MIN_ARG))).astype(F32)
     d = F32(1.0) + e
     q = recip_1_2(d)
     sigma = np.where(t >= 0, q, e * q).astype(F32)

@@ -1,5 +1,6 @@
 """Pins of the oracle's GELU and MLP chain (oracle/mlp.py) against values fixed by mathematics."""
 import math
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -16,15 +17,55 @@ def _all_finite_bf16() -> np.ndarray:
     return y[np.isfinite(y)]
 
 
+def _round_fraction_to_f32(x: Fraction) -> float:
+    """Exact round-to-nearest-even of a rational to binary32 (normal and subnormal range)."""
+    if x == 0:
+        return 0.0
+    sign = -1 if x < 0 else 1
+    x = abs(x)
+    e = x.numerator.bit_length() - x.denominator.bit_length()      # 2^(e-1) < x < 2^(e+1)
+    while Fraction(2) ** e <= x:
+        e += 1
+    while Fraction(2) ** (e - 1) > x:
+        e -= 1                                                       # 2^(e-1) <= x < 2^e
+    q = max(e - 24, -149)                                            # spacing 2^q
+    m = x / Fraction(2) ** q
+    n = m.numerator // m.denominator
+    rem = m - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return sign * float(Fraction(n) * Fraction(2) ** q)
+
+
+def test_fma32_is_one_rounding_of_the_exact_value():
+    rng = np.random.default_rng(3)
+    a = rng.standard_normal(3000).astype(np.float32) * np.float32(3.0)
+    b = rng.standard_normal(3000).astype(np.float32)
+    c = rng.standard_normal(3000).astype(np.float32) * np.float32(0.5)
+    # products whose low bits make a + b*c land on (or next to) binary32 midpoints
+    k = np.arange(1, 400, dtype=np.float32)
+    a2 = (np.float32(1.0) + k * np.float32(2.0 ** -12)).astype(np.float32)
+    b2 = (np.float32(1.0) + np.float32(2.0 ** -12)) * np.ones_like(a2)
+    c2 = np.where(np.arange(k.size) % 3 == 0, np.float32(2.0 ** -60),
+                  np.where(np.arange(k.size) % 3 == 1, np.float32(-2.0 ** -60), np.float32(0.0))).astype(np.float32)
+    tiny = np.array([1e-40, -1e-40, 3e-39], dtype=np.float32)          # subnormal results
+    for A, B, Cc in ((a, b, c), (a2, b2, c2), (tiny, np.float32([0.5, 0.75, 1.5]), np.float32([1e-45, 0.0, -1e-45]))):
+        got = OM.fma32(A, B, Cc)
+        for i in range(A.size):
+            exact = Fraction(float(A[i])) * Fraction(float(B[i])) + Fraction(float(Cc[i]))
+            assert float(got[i]) == _round_fraction_to_f32(exact), (A[i], B[i], Cc[i])
+
+
 def test_exp_against_float64_exponential():
     x = -np.linspace(0.0, 80.0, 400001).astype(np.float32)
-    e = OM.exp_nonpos_f32(x).astype(np.float64)
+    e = OM.exp_m80_0_f32(x).astype(np.float64)
     ref = np.exp(x.astype(np.float64))
-    assert np.max(np.abs(e - ref) / ref) <= 2.5 * 2.0 ** -24     # within 2.5 ulp of float32
-    assert OM.exp_nonpos_f32(np.float32(0.0)) == 1.0
-    assert OM.exp_nonpos_f32(np.float32(-80.5)) == 0.0         # below the cut-off
+    assert np.max(np.abs(e - ref) / ref) <= 4.0 * 2.0 ** -24     # within 4 ulp of float32
+    assert OM.exp_m80_0_f32(np.float32(0.0)) == 1.0
     with pytest.raises(ValueError):
-        OM.exp_nonpos_f32(np.float32(1.0))
+        OM.exp_m80_0_f32(np.float32(1.0))
+    with pytest.raises(ValueError):
+        OM.exp_m80_0_f32(np.float32(-80.5))
 
 
 def test_reciprocal_on_one_to_two():
@@ -39,6 +80,7 @@ def test_reciprocal_on_one_to_two():
 def test_taylor_coefficients_are_reciprocal_factorials():
     for k, c in enumerate(OM.TAYLOR):
         assert c == np.float32(1.0 / math.factorial(k))
+    assert OM.C3 == np.float32(float(OM.C2) * 0.044715) or abs(float(OM.C3) / (float(OM.C2) * 0.044715) - 1) < 1e-7
     assert float(OM.LN2_HI) + float(OM.LN2_LO) == pytest.approx(math.log(2.0), rel=1e-15, abs=1e-12)
     assert float(OM.LN2_HI) * 65536.0 == int(float(OM.LN2_HI) * 65536.0)    # 16 significant bits
 
@@ -50,8 +92,8 @@ def test_gelu_f32_against_logistic_form_on_every_bf16_input():
     with np.errstate(over="ignore"):
         t = np.abs(2.0 * np.sqrt(2.0 / np.pi) * (y.astype(np.float64) + 0.044715 * y.astype(np.float64) ** 3))
     # exp(-|t|) turns the relative rounding of t into |t| times as much: the bound grows with |t|;
-    # below exp(-80) the result is cut to zero (|GELU| < 2e-33 there).
-    bound = 4.0 * 2.0 ** -24 * (2.0 + np.minimum(t, 1e30)) * np.abs(c) + 2e-33
+    # below exp(-80) the exponential is cut to zero (|GELU| < 2e-33 there).
+    bound = 6.0 * 2.0 ** -24 * (2.0 + np.minimum(t, 1e30)) * np.abs(c) + 2e-33
     assert np.all(np.abs(g - c) <= bound)
 
 
