@@ -69,7 +69,8 @@ constexpr int LN_SMEM = LN_OFF_BAR + 256 + 1024;
 // read back by ldmatrix; a warp pair's 2 KB also carries the pair's partial-sum hand-off).
 constexpr int LN_OFF_STG = LN_OFF_BAR + 256;
 constexpr int LN_STG_BYTES = 1024;
-constexpr int LN_SMEM_GQ = LN_OFF_STG + LN_EPI_WARPS * LN_STG_BYTES + 1024;
+constexpr int LN_OFF_RCP = LN_OFF_STG + LN_EPI_WARPS * LN_STG_BYTES;   // 256 floats: f32(1/f32(dec(sb) gs2))
+constexpr int LN_SMEM_GQ = LN_OFF_RCP + 1024 + 1024;
 constexpr int LN_GQ_MAX_R = 32;
 static_assert(LN_SMEM_GQ <= 232448, "shared memory budget of the fused epilogue");
 constexpr uint64_t LN_DEFAULT_TIMEOUT_NS = 2000000000ull;
@@ -297,6 +298,12 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (GQ && threadIdx.x < 256) {
+    // The next layer's quantizer: rinv = f32(1 / f32(dec(sb) gs2)) for every UE4M3 byte (0 for sb = 0).
+    float* rcp = reinterpret_cast<float*>(smem + LN_OFF_RCP);
+    const uint32_t sb = threadIdx.x;
+    rcp[sb] = sb ? __frcp_rn(__fmul_rn(dec_ue4m3(sb), args.gs_x2)) : 0.0f;
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, LN_TMEM_COLS);
@@ -545,6 +552,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
     const int KS4 = N >> 6;                          // scale words per row of the next layer
     const uint32_t stg = smem_u32(smem + LN_OFF_STG + (2 * q + h) * LN_STG_BYTES);
     const uint32_t pairbuf = smem_u32(smem + LN_OFF_STG + 2 * q * LN_STG_BYTES);
+    const uint32_t rcp_tab = smem_u32(smem + LN_OFF_RCP);
     const int gid = lane >> 2, tig = lane & 3;
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
@@ -568,7 +576,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
       const int row = mb * LN_BM + 32 * q + lane;
       const int n0 = nb * LN_BN + h * 128;
       uint32_t p[64];                                // y, then x2 (bf16 pairs): p[8g + j] = columns 16g + 2j, +1
-      uint32_t cw[16];                               // codes: two words per group of 16
+      uint32_t cw[4];                                // codes of two groups of 16 (two words each)
       uint32_t sw[2] = {0u, 0u};                     // scale words (4 groups each)
       // y = f32(gs acc + bias) rounded to bf16, as bf16 pairs (the accumulator registers end here,
       // which leaves room for the GELU of several pairs at a time)
@@ -611,7 +619,7 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
                              fmaxf(fabsf(xh[2 * k + 1].x), fabsf(xh[2 * k + 1].y))));
         }
         const uint32_t sb = valid ? cvt_ue4m3(__fmul_rn(a, c_x2)) : 0u;
-        const float rinv = sb ? __frcp_rn(__fmul_rn(dec_ue4m3(sb), gs2)) : 0.0f;
+        const float rinv = lds_f32(rcp_tab + 4 * sb);
         const float2 rr = make_float2(rinv, rinv);
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
@@ -622,15 +630,12 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
             qv[2 * i] = q2.x;
             qv[2 * i + 1] = q2.y;
           }
-          cw[2 * g + hb] = sb ? cvt_e2m1x8(qv) : 0u;
+          cw[2 * (g & 1) + hb] = sb ? cvt_e2m1x8(qv) : 0u;
         }
+        if ((g & 1) && row < M && n0 + 16 * (g - 1) < N)    // codes of groups g-1, g: 16 bytes
+          reinterpret_cast<uint4*>(args.Xq2 + (int64_t)row * (N >> 1) + (n0 >> 1))[g >> 1] =
+              make_uint4(cw[0], cw[1], cw[2], cw[3]);
         sw[g >> 2] |= sb << (8 * (g & 3));
-      }
-      if (row < M) {
-        uint4* dst = reinterpret_cast<uint4*>(args.Xq2 + (int64_t)row * (N >> 1) + (n0 >> 1));
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (n0 + 32 * u < N) dst[u] = make_uint4(cw[4 * u], cw[4 * u + 1], cw[4 * u + 2], cw[4 * u + 3]);
       }
 #pragma unroll
       for (int kw = 0; kw < 2; ++kw)          // padding rows (M .. Mpad) hold zero scales

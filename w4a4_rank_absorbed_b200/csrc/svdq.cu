@@ -512,8 +512,8 @@ svdq_status svdq_gelu_bf16(const uint16_t* X, int64_t n, uint16_t* Y, svdq_strea
   svdq_status st;
   if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
   const int64_t nv = (n + 7) / 8;
-  const int64_t cap = (int64_t)d->sms * 8;
-  const int blocks = (int)std::min<int64_t>((nv + 255) / 256, cap);
+  const int64_t cap = (int64_t)d->sms * 8;                   // 8 blocks of 256 threads per SM
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nv + 4 * 256 - 1) / (4 * 256), cap));
   if (launch_pdl(k_gelu_bf16, dim3(blocks), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), 1, X, n, Y) !=
       cudaSuccess)
     return SVDQ_ERR_CUDA;
