@@ -337,6 +337,36 @@ SVDQ_API svdq_status svdq_linear_gelu_quantize(const uint8_t* Xq, const uint8_t*
 SVDQ_API svdq_status svdq_gelu_bf16(const uint16_t* X, int64_t n, uint16_t* Y, svdq_stream_t stream);
 
 /*
+ * Calibration on the GPU ("From SmoothQuant to SVDQuant", quantization scheme:
+ * the smoothing factors, the low-rank split and the activation global scale are
+ * fixed offline from calibration data; section Smooth Quant (W8A8): the
+ * per-channel factor s_j = max|X_j|^alpha / max|W_j|^(1 - alpha)).  These calls
+ * compute the statistics and the smoothing; the truncated SVD of W_hat is done
+ * by the caller (the Python layer uses a randomized range finder on the GPU).
+ * Every maximum is exact (maxima merge by an order-independent atomic max).
+ *
+ * svdq_calib_absmax_cols: amax_x[j] = max over rows of |X[m, j]|, X bf16 M x K
+ *   (K % 8 == 0, X 16-byte aligned).  accumulate = 1 merges into amax_x (max with
+ *   its contents: several calibration batches in turn), 0 starts from zero.
+ * svdq_calib_absmax_rows: amax_w[j] = max over n of |W[j, n]|, W float64 K x N.
+ * svdq_calib_smooth: s_j = amax_x[j]^alpha / amax_w[j]^(1 - alpha) in float64
+ *   (1 where either maximum is 0), inv_s[j] = f32(1 / s_j); 0 <= alpha <= 1.
+ * svdq_calib_scale_rows: W_hat = diag(s) W, float64 K x N (one rounding each).
+ * svdq_calib_act_amax: amax = max |f32(X * inv_s)| over a bf16 M x K X (the
+ *   activation global scale is f32(amax / 2688)); accumulate as above.
+ */
+SVDQ_API svdq_status svdq_calib_absmax_cols(const uint16_t* X, int64_t M, int64_t K, float* amax_x, int accumulate,
+                                            svdq_stream_t stream);
+SVDQ_API svdq_status svdq_calib_absmax_rows(const double* W, int64_t K, int64_t N, double* amax_w,
+                                            svdq_stream_t stream);
+SVDQ_API svdq_status svdq_calib_smooth(const float* amax_x, const double* amax_w, int64_t K, double alpha,
+                                       double* s, float* inv_s, svdq_stream_t stream);
+SVDQ_API svdq_status svdq_calib_scale_rows(const double* W, const double* s, int64_t K, int64_t N, double* W_hat,
+                                           svdq_stream_t stream);
+SVDQ_API svdq_status svdq_calib_act_amax(const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float* amax,
+                                         int accumulate, svdq_stream_t stream);
+
+/*
  * svdq_lowrank_down -- the low-rank down-projection as a kernel of its own: the
  * unfused form of the branch (SVDQuant review, §4.3: without fusion the branch
  * re-reads the 16-bit activations from memory, which is what the fused

@@ -46,3 +46,21 @@ def test_calibration_matches_the_oracle(case):
     assert np.linalg.norm(LL_got - LL_or) / np.linalg.norm(LL_or) <= 1e-3
     if wl.bias is not None:
         assert np.array_equal(got.bias.float().numpy(), torch.from_numpy(wl.bias).to(torch.bfloat16).float().numpy())
+
+
+def test_randomized_range_finder_on_cpu_matches_truncated_svd():
+    """The randomized split (the GPU calibration's algorithm; torch on the CPU here) against numpy's
+    truncated SVD: same error to 1e-3 and the same leading singular values."""
+    import torch
+    from oracle import decompose as OD
+    from w4a4_rank_absorbed_b200.calib import randomized_rank_r
+    from w4a4_rank_absorbed_b200.synth import make_workload
+    wl = make_workload("tiny")
+    s = OD.smoothing_factors(wl.X, wl.W, wl.alpha)
+    W_hat = s[:, None] * wl.W
+    _, _, R, S = OD.low_rank_split(W_hat, 32)
+    G1, G2 = randomized_rank_r(torch.from_numpy(W_hat), 32)
+    err = float(torch.linalg.norm(torch.from_numpy(W_hat) - G1 @ G2))
+    assert err <= np.linalg.norm(R) * (1 + 1e-3)
+    sg = torch.linalg.svdvals(G1 @ G2).numpy()[:4]
+    assert np.max(np.abs(sg - S[:4]) / S[:4]) <= 1e-8

@@ -125,3 +125,76 @@ def calibrate(X, W, r: int, alpha: float = 0.5, bias=None, lora_A=None, lora_B=N
     return LayerData(K=K, N=N, r=L1.shape[1], inv_s=inv_s, gs_x=act_global_scale(Xc, inv_s),
                      L1fT=L1fT, L2b=L2.contiguous().to(torch.bfloat16), R=R.to(torch.float32).contiguous(),
                      bias=None if bias is None else _as64(bias).to(torch.bfloat16), s=s)
+
+
+# ------------------------------------------------------------------ on the GPU --
+def randomized_rank_r(W_hat: torch.Tensor, r: int, oversample: int = 32, power_iters: int = 6,
+                      seed: int = 0):
+    """Rank-r factors (L1 = U_r Sigma_r, L2 = V_r^T) of a float64 K x N matrix on its device by a
+    randomized range finder: Y = W_hat Omega (Omega Gaussian N x (r + oversample)), power_iters
+    rounds of Y = W_hat (W_hat^T Q) with re-orthonormalization, then the exact SVD of the small
+    B = Q^T W_hat.  The products are library float64 GEMMs and the orthonormalizations library QR
+    factorizations (offline, outside the layer's forward pass)."""
+    K, N = W_hat.shape
+    ell = min(r + oversample, K, N)
+    g = torch.Generator(device=W_hat.device).manual_seed(seed)
+    Omega = torch.randn((N, ell), dtype=torch.float64, device=W_hat.device, generator=g)
+    Q, _ = torch.linalg.qr(W_hat @ Omega)
+    for _ in range(power_iters):
+        Z, _ = torch.linalg.qr(W_hat.T @ Q)
+        Q, _ = torch.linalg.qr(W_hat @ Z)
+    B = Q.T @ W_hat
+    Ub, S, Vh = torch.linalg.svd(B, full_matrices=False)
+    U = Q @ Ub
+    return U[:, :r] * S[:r][None, :], Vh[:r, :]
+
+
+def calibrate_gpu(X, W, r: int, alpha: float = 0.5, bias=None, lora_A=None, lora_B=None, X_cal=None,
+                  device=None, oversample: int = 32, power_iters: int = 6, seed: int = 0,
+                  batch_rows: int = 8192) -> LayerData:
+    """calibrate() with its statistics and its split on the GPU.
+
+    Activation channel maxima stream over the calibration rows in batches (svdq_calib_absmax_cols,
+    merged by max), weight channel maxima, smoothing factors and W_hat = diag(s) W come from the
+    library's calibration kernels (float64 for everything weight-side), the rank-r split from
+    randomized_rank_r, and gs_x from the maximum of f32(X * inv_s) (svdq_calib_act_amax).  The
+    maxima, s and W_hat are those of calibrate(); the split differs from the exact truncated SVD only
+    by the randomized range finder's approximation."""
+    from . import svdq as C
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    Xc = X if X_cal is None else X_cal
+    Xc = Xc if isinstance(Xc, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(Xc, dtype=np.float32))
+    Wd = _as64(W)
+    K, N = Wd.shape
+    with torch.cuda.device(dev):
+        Xb = Xc.to(torch.bfloat16)
+        amax_x = torch.empty(K, dtype=torch.float32, device=dev)
+        M = Xb.shape[0]
+        for i, lo in enumerate(range(0, max(M, 1), batch_rows)):
+            xb = Xb[lo:lo + batch_rows].to(dev).contiguous()
+            C.svdq_calib_absmax_cols(xb, xb.shape[0], K, amax_x, accumulate=i > 0)
+        W_dev = Wd.to(dev).contiguous()
+        amax_w = torch.empty(K, dtype=torch.float64, device=dev)
+        C.svdq_calib_absmax_rows(W_dev, K, N, amax_w)
+        s = torch.empty(K, dtype=torch.float64, device=dev)
+        inv_s = torch.empty(K, dtype=torch.float32, device=dev)
+        C.svdq_calib_smooth(amax_x, amax_w, K, alpha, s, inv_s)
+        W_hat = torch.empty_like(W_dev)
+        C.svdq_calib_scale_rows(W_dev, s, K, N, W_hat)
+        del W_dev
+        L1, L2 = randomized_rank_r(W_hat, r, oversample, power_iters, seed)
+        R = torch.addmm(W_hat, L1, L2, alpha=-1.0)
+        del W_hat
+        if lora_A is not None:
+            L1 = torch.cat([L1, s[:, None] * _as64(lora_A).to(dev)], dim=1)
+            L2 = torch.cat([L2, _as64(lora_B).to(dev)], dim=0)
+        amax = torch.empty(1, dtype=torch.float32, device=dev)
+        for i, lo in enumerate(range(0, max(M, 1), batch_rows)):
+            xb = Xb[lo:lo + batch_rows].to(dev).contiguous()
+            C.svdq_calib_act_amax(xb, xb.shape[0], K, inv_s, amax, accumulate=i > 0)
+        a = float(amax.item())
+        gs_x = 1.0 if a == 0.0 else float(np.float32(np.float64(a) / 2688.0))
+        L1fT = (L1 / s[:, None]).t().contiguous().to(torch.bfloat16)
+        return LayerData(K=K, N=N, r=L1.shape[1], inv_s=inv_s.cpu(), gs_x=gs_x, L1fT=L1fT.cpu(),
+                         L2b=L2.contiguous().to(torch.bfloat16).cpu(), R=R.to(torch.float32).contiguous().cpu(),
+                         bias=None if bias is None else _as64(bias).to(torch.bfloat16), s=s.cpu())

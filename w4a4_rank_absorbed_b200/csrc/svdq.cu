@@ -14,6 +14,7 @@
 
 #include "../../include/svdq.h"
 #include "common.cuh"
+#include "calib.cuh"
 #include "linear.cuh"
 #include "pack_weight.cuh"
 #include "quantize_act.cuh"
@@ -517,6 +518,83 @@ svdq_status svdq_gelu_bf16(const uint16_t* X, int64_t n, uint16_t* Y, svdq_strea
   if (launch_pdl(k_gelu_bf16, dim3(blocks), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), 1, X, n, Y) !=
       cudaSuccess)
     return SVDQ_ERR_CUDA;
+  return launch_status();
+}
+
+svdq_status svdq_calib_absmax_cols(const uint16_t* X, int64_t M, int64_t K, float* amax_x, int accumulate,
+                                   svdq_stream_t stream) {
+  if (M < 0 || K < 8 || K % 8 != 0 || K >= (int64_t(1) << 31) || !amax_x || (M > 0 && !X) ||
+      (accumulate != 0 && accumulate != 1))
+    return SVDQ_ERR_INVALID_ARG;
+  if ((M > 0 && !aligned16(X)) || (reinterpret_cast<uintptr_t>(amax_x) & 3u)) return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  svdq_status st;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!accumulate && cudaMemsetAsync(amax_x, 0, (size_t)K * sizeof(float), s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (M == 0) return launch_status();
+  const int gx = (int)((K + 255) / 256);
+  // enough row slices for about four blocks per SM
+  const int64_t want = std::max<int64_t>(1, (int64_t)d->sms * 4 / gx);
+  const int slices = (int)std::min<int64_t>(want, (M + 63) / 64);
+  const int rows = (int)((M + slices - 1) / slices);
+  k_absmax_cols<<<dim3(gx, (unsigned)((M + rows - 1) / rows)), 256, 0, s>>>(X, M, (int)K, rows, amax_x);
+  return launch_status();
+}
+
+svdq_status svdq_calib_absmax_rows(const double* W, int64_t K, int64_t N, double* amax_w, svdq_stream_t stream) {
+  if (K < 1 || N < 1 || K >= (int64_t(1) << 31) || !W || !amax_w) return SVDQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(amax_w)) & 7u) return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  svdq_status st;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  k_absmax_rows<<<(unsigned)K, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, N, amax_w);
+  return launch_status();
+}
+
+svdq_status svdq_calib_smooth(const float* amax_x, const double* amax_w, int64_t K, double alpha, double* s,
+                              float* inv_s, svdq_stream_t stream) {
+  if (K < 1 || K >= (int64_t(1) << 31) || !amax_x || !amax_w || !s || !inv_s || !(alpha >= 0.0 && alpha <= 1.0))
+    return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  DevInfo* d;
+  svdq_status st;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  k_smooth<<<(unsigned)((K + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(amax_x, amax_w, (int)K,
+                                                                                           alpha, s, inv_s);
+  return launch_status();
+}
+
+svdq_status svdq_calib_scale_rows(const double* W, const double* s, int64_t K, int64_t N, double* W_hat,
+                                  svdq_stream_t stream) {
+  if (K < 1 || N < 1 || !W || !s || !W_hat) return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  DevInfo* d;
+  svdq_status st;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  const int64_t blocks = std::min<int64_t>((K * N + 255) / 256, (int64_t)d->sms * 16);
+  k_scale_rows<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, s, K, N, W_hat);
+  return launch_status();
+}
+
+svdq_status svdq_calib_act_amax(const uint16_t* X, int64_t M, int64_t K, const float* inv_s, float* amax,
+                                int accumulate, svdq_stream_t stream) {
+  if (M < 0 || K < 8 || K % 8 != 0 || K >= (int64_t(1) << 31) || !inv_s || !amax || (M > 0 && !X) ||
+      (accumulate != 0 && accumulate != 1))
+    return SVDQ_ERR_INVALID_ARG;
+  if ((M > 0 && !aligned16(X)) || !aligned16(inv_s) || (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return SVDQ_ERR_MISALIGNED;
+  int dev;
+  DevInfo* d;
+  svdq_status st;
+  if ((st = current_device(&dev, &d)) != SVDQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!accumulate && cudaMemsetAsync(amax, 0, sizeof(float), s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (M == 0) return launch_status();
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((M * (K / 8) + 255) / 256, (int64_t)d->sms * 8));
+  k_act_amax<<<(unsigned)blocks, 256, 0, s>>>(X, M, (int)K, inv_s, amax);
   return launch_status();
 }
 

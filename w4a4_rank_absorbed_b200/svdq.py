@@ -30,7 +30,9 @@ EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_we
             "svdq_linear", "svdq_lowrank_down", "svdq_lowrank_up", "svdq_get_device_error", "svdq_linear_debug",
             "svdq_quantize_act_workspace_bytes", "svdq_dequant_weight", "svdq_quantize_act_noalloc",
             "svdq_mx_sf_bytes", "svdq_pack_weight_mx", "svdq_quantize_act_mx", "svdq_linear_mx",
-            "svdq_linear_gelu_quantize", "svdq_linear_gelu_quantize_workspace_bytes", "svdq_gelu_bf16")
+            "svdq_linear_gelu_quantize", "svdq_linear_gelu_quantize_workspace_bytes", "svdq_gelu_bf16",
+            "svdq_calib_absmax_cols", "svdq_calib_absmax_rows", "svdq_calib_smooth", "svdq_calib_scale_rows",
+            "svdq_calib_act_amax")
 
 
 class SVDQError(RuntimeError):
@@ -95,6 +97,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                               _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
     lib.svdq_gelu_bf16.restype = _I
     lib.svdq_gelu_bf16.argtypes = [_P, _I64, _P, _P]
+    _D = ctypes.c_double
+    for name, args in (("svdq_calib_absmax_cols", [_P, _I64, _I64, _P, _I, _P]),
+                       ("svdq_calib_absmax_rows", [_P, _I64, _I64, _P, _P]),
+                       ("svdq_calib_smooth", [_P, _P, _I64, _D, _P, _P, _P]),
+                       ("svdq_calib_scale_rows", [_P, _P, _I64, _I64, _P, _P]),
+                       ("svdq_calib_act_amax", [_P, _I64, _I64, _P, _P, _I, _P])):
+        getattr(lib, name).restype = _I
+        getattr(lib, name).argtypes = args
     lib.svdq_get_device_error.restype = _I
     lib.svdq_get_device_error.argtypes = [_P, ctypes.POINTER(_I)]
     _lib = lib
@@ -205,6 +215,34 @@ def svdq_gelu_bf16(X, n, Y, stream=None) -> None:
     lib = load_library()
     st = lib.svdq_gelu_bf16(_ptr(X, torch.bfloat16, "X"), n, _ptr(Y, torch.bfloat16, "Y"), _stream(stream))
     _check(st, "svdq_gelu_bf16")
+
+
+def svdq_calib_absmax_cols(X, M, K, amax_x, accumulate=False, stream=None) -> None:
+    _check(load_library().svdq_calib_absmax_cols(_ptr(X, torch.bfloat16, "X"), M, K, _ptr(amax_x, torch.float32, "amax_x"),
+                                                 int(bool(accumulate)), _stream(stream)), "svdq_calib_absmax_cols")
+
+
+def svdq_calib_absmax_rows(W, K, N, amax_w, stream=None) -> None:
+    _check(load_library().svdq_calib_absmax_rows(_ptr(W, torch.float64, "W"), K, N, _ptr(amax_w, torch.float64, "amax_w"),
+                                                 _stream(stream)), "svdq_calib_absmax_rows")
+
+
+def svdq_calib_smooth(amax_x, amax_w, K, alpha, s, inv_s, stream=None) -> None:
+    _check(load_library().svdq_calib_smooth(_ptr(amax_x, torch.float32, "amax_x"), _ptr(amax_w, torch.float64, "amax_w"),
+                                            K, float(alpha), _ptr(s, torch.float64, "s"),
+                                            _ptr(inv_s, torch.float32, "inv_s"), _stream(stream)), "svdq_calib_smooth")
+
+
+def svdq_calib_scale_rows(W, s, K, N, W_hat, stream=None) -> None:
+    _check(load_library().svdq_calib_scale_rows(_ptr(W, torch.float64, "W"), _ptr(s, torch.float64, "s"), K, N,
+                                                _ptr(W_hat, torch.float64, "W_hat"), _stream(stream)),
+           "svdq_calib_scale_rows")
+
+
+def svdq_calib_act_amax(X, M, K, inv_s, amax, accumulate=False, stream=None) -> None:
+    _check(load_library().svdq_calib_act_amax(_ptr(X, torch.bfloat16, "X"), M, K, _ptr(inv_s, torch.float32, "inv_s"),
+                                              _ptr(amax, torch.float32, "amax"), int(bool(accumulate)),
+                                              _stream(stream)), "svdq_calib_act_amax")
 
 
 def svdq_version() -> int:
