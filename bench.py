@@ -70,6 +70,9 @@ def parse(argv=None):
     p.add_argument("--cpu-sample-rows", type=int, default=0, help="oracle rows (0 = every row of the batch)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--profile-case", action="store_true",
+                   help="run each kernel of the step once on one copy of the headline layer, then the fused "
+                        "fc1 GEMM of the MLP pair once, and exit (the case the ncu captures are taken on)")
     return p.parse_args(argv)
 
 
@@ -707,8 +710,46 @@ def pack_leg(data, dev, timer):
             "note": "offline, once per layer; not in the step"}
 
 
+def run_profile_case(args):
+    """One launch of each kernel on one layer copy (calibrated on the GPU), few launches in all: the
+    small case the full ncu captures are taken on.  Device memory: a few hundred MB."""
+    import torch
+
+    from w4a4_rank_absorbed_b200 import build
+    build.build()
+    from w4a4_rank_absorbed_b200 import svdq as C
+    from w4a4_rank_absorbed_b200.calib import calibrate_gpu
+    from w4a4_rank_absorbed_b200.layer import SVDQLinear
+    from w4a4_rank_absorbed_b200.synth import make_workload
+    dev = torch.device("cuda", 0)
+    wl = make_workload(args.workload)
+    L = SVDQLinear(calibrate_gpu(wl.X, wl.W, wl.r, wl.alpha, bias=wl.bias, device=dev), device=dev)
+    X = torch.from_numpy(wl.X.astype(np.float32)).to(torch.bfloat16).to(dev)
+    Y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
+    L.gemm(*L.quantize(X), Y)
+    torch.cuda.synchronize()
+    del L, X, Y
+    w1, w2 = make_workload("fc1"), make_workload("fc2")
+    X1 = torch.from_numpy(w1.X.astype(np.float32)).to(torch.bfloat16).to(dev)
+    L1 = SVDQLinear(calibrate_gpu(w1.X, w1.W, w1.r, w1.alpha, bias=w1.bias, device=dev), device=dev)
+    X2 = torch.empty((w1.M, w1.N), dtype=torch.bfloat16, device=dev)
+    Y1 = L1.forward(X1)
+    C.svdq_gelu_bf16(Y1, Y1.numel(), X2)
+    L2 = SVDQLinear(calibrate_gpu(X2.float().cpu(), w2.W, w2.r, w2.alpha, bias=w2.bias, device=dev), device=dev)
+    del Y1
+    L1.gemm_gelu_quantize(*L1.quantize(X1), L2)
+    torch.cuda.synchronize()
+    st, site = C.svdq_get_device_error()
+    if st != 0:
+        raise SystemExit(f"device error {st} at {site:#x}")
+    print("profile case done", flush=True)
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        run_profile_case(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
