@@ -401,6 +401,16 @@ SVDQ_API svdq_status svdq_lowrank_up(const uint16_t* LAs, const uint16_t* L2p, i
                             int64_t M, int64_t N, svdq_stream_t stream);
 
 /*
+ * svdq_map_cache_stats -- counters of the library's host cache of TMA tensor
+ * maps (64 entries, keyed by address, element type, shape, strides, box and
+ * swizzle; least recently used replaced): a call whose buffers and shapes were
+ * seen before reuses the encoded maps instead of encoding them again.  The
+ * pages have no counterpart (it is host-side launch cost).  hits / misses may
+ * be NULL.
+ */
+SVDQ_API void svdq_map_cache_stats(uint64_t* hits, uint64_t* misses);
+
+/*
  * svdq_get_device_error -- synchronises `stream`, then reads and clears the
  * library's device error word on the current device.  Returns SVDQ_OK, or
  * SVDQ_ERR_TIMEOUT when a kernel's bounded wait on a barrier ran out (the

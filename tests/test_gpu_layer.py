@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import OL, check_y, require_gpu
+from helpers import OL, GpuLayer, bf16_dev, check_y, oracle_layer, require_gpu
 from w4a4_rank_absorbed_b200.synth import small_case
 
 pytestmark = pytest.mark.gpu
@@ -61,3 +61,29 @@ def test_streamed_host_batches_match_forward():
         assert torch.equal(Yh[i], want[i]), f"batch {i}"
     from w4a4_rank_absorbed_b200 import svdq as C
     assert C.svdq_get_device_error()[0] == 0
+
+
+def test_tensor_maps_are_cached_across_calls():
+    """The second and later forward passes on the same buffers encode no tensor map; host time per call
+    through the C ABI is printed (eager launches, no graph)."""
+    import time
+    from w4a4_rank_absorbed_b200 import svdq as C
+    wl = small_case(256, 512, 512, 32, seed=5)
+    dec = oracle_layer(wl, 32)
+    g = GpuLayer(dec, wl.bias)
+    X = bf16_dev(wl.X)
+    Xq, SFx, LAs = g.quantize(X)
+    Y = g.linear(Xq, SFx, LAs)
+    torch.cuda.synchronize()
+    h0, m0 = C.svdq_map_cache_stats()
+    n = 200
+    t0 = time.perf_counter()
+    for _ in range(n):
+        C.svdq_linear(Xq, SFx, float(g.gs_x), g.Wq, g.SFw, float(g.gs_w), LAs, g.L2p, g.r, g.bias, Y, 0, 256, 512, 512)
+    t1 = time.perf_counter()
+    torch.cuda.synchronize()
+    h1, m1 = C.svdq_map_cache_stats()
+    assert m1 == m0, "a repeated call encoded a tensor map again"
+    assert h1 - h0 == 4 * n                      # Xq, Wq, LAs, L2p maps of every call
+    print(f"svdq_linear host time per call through ctypes, cached maps: {(t1 - t0) / n * 1e6:.1f} us")
+    g.check_errors()

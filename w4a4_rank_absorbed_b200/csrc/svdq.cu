@@ -78,33 +78,105 @@ EncodeTiledFn encode_fn() {
 
 // 2-D row-major tensor (rows x inner elements, row pitch in bytes), box (box_inner x box_rows),
 // 128-byte swizzle unless stated.
+// Tensor maps are cached on the host: a call on the same buffers with the same shapes (every forward
+// pass of a layer) reuses the encoded map instead of encoding it again.  A map holds only the
+// address, the shape and the box, so a cached entry stays valid for any later buffer at the same
+// address with the same shape.  64 entries, least recently used replaced, one mutex.
+struct MapKey {
+  const void* base;
+  uint32_t dt, rank, swizzle;
+  uint64_t dims[3], strides[2];
+  uint32_t box[3];
+  bool operator==(const MapKey& o) const {
+    return base == o.base && dt == o.dt && rank == o.rank && swizzle == o.swizzle &&
+           std::memcmp(dims, o.dims, sizeof(dims)) == 0 && std::memcmp(strides, o.strides, sizeof(strides)) == 0 &&
+           std::memcmp(box, o.box, sizeof(box)) == 0;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  uint64_t stamp = 0;
+  bool used = false;
+};
+constexpr int kMapCacheEntries = 64;
+MapEntry g_maps[kMapCacheEntries];
+uint64_t g_map_clock = 0;
+uint64_t g_map_hits = 0, g_map_misses = 0;
+std::mutex g_map_mu;
+
+bool encode_map(const MapKey& k, CUtensorMap* m) {
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (MapEntry& e : g_maps)
+      if (e.used && e.key == k) {
+        e.stamp = ++g_map_clock;
+        *m = e.map;
+        ++g_map_hits;
+        return true;
+      }
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {k.dims[0], k.dims[1], k.dims[2]};
+  cuuint64_t strides[2] = {k.strides[0], k.strides[1]};
+  cuuint32_t box[3] = {k.box[0], k.box[1], k.box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (fn(m, (CUtensorMapDataType)k.dt, k.rank, const_cast<void*>(k.base), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)k.swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  MapEntry* victim = &g_maps[0];
+  for (MapEntry& e : g_maps) {
+    if (!e.used) {
+      victim = &e;
+      break;
+    }
+    if (e.stamp < victim->stamp) victim = &e;
+  }
+  victim->key = k;
+  victim->map = *m;
+  victim->stamp = ++g_map_clock;
+  victim->used = true;
+  ++g_map_misses;
+  return true;
+}
+
 bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
                  uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows,
                  CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {pitch_bytes};
-  cuuint32_t box[2] = {box_inner, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  MapKey k{};
+  k.base = base;
+  k.dt = (uint32_t)dt;
+  k.rank = 2;
+  k.swizzle = (uint32_t)swizzle;
+  k.dims[0] = inner;
+  k.dims[1] = rows;
+  k.strides[0] = pitch_bytes;
+  k.box[0] = box_inner;
+  k.box[1] = box_rows;
+  return encode_map(k, m);
 }
 
 // The rows x K bf16 matrix at `base` as a 3-D tensor {64 columns, rows, K/64 chunks} (strides 2K and
 // 128 bytes), box {64, box_rows, 2}, 128-byte swizzle: one copy brings two adjacent 64-column
 // chunks of box_rows rows and lands them as two 128-byte-swizzled tiles, one after the other.
 bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {64, rows, K / 64};
-  cuuint64_t strides[2] = {K * 2, 128};
-  cuuint32_t box[3] = {64, box_rows, 2};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  MapKey k{};
+  k.base = base;
+  k.dt = (uint32_t)CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  k.rank = 3;
+  k.swizzle = (uint32_t)CU_TENSOR_MAP_SWIZZLE_128B;
+  k.dims[0] = 64;
+  k.dims[1] = rows;
+  k.dims[2] = K / 64;
+  k.strides[0] = K * 2;
+  k.strides[1] = 128;
+  k.box[0] = 64;
+  k.box[1] = box_rows;
+  k.box[2] = 2;
+  return encode_map(k, m);
 }
 
 // ------------------------------------------------------------- checks -------
@@ -596,6 +668,12 @@ svdq_status svdq_calib_act_amax(const uint16_t* X, int64_t M, int64_t K, const f
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((M * (K / 8) + 255) / 256, (int64_t)d->sms * 8));
   k_act_amax<<<(unsigned)blocks, 256, 0, s>>>(X, M, (int)K, inv_s, amax);
   return launch_status();
+}
+
+void svdq_map_cache_stats(uint64_t* hits, uint64_t* misses) {
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (hits) *hits = g_map_hits;
+  if (misses) *misses = g_map_misses;
 }
 
 svdq_status svdq_dequant_weight(const uint8_t* Wq, const uint8_t* SFw, const float* gs_w, int64_t K, int64_t N,

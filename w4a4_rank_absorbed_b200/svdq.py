@@ -32,7 +32,7 @@ EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_we
             "svdq_mx_sf_bytes", "svdq_pack_weight_mx", "svdq_quantize_act_mx", "svdq_linear_mx",
             "svdq_linear_gelu_quantize", "svdq_linear_gelu_quantize_workspace_bytes", "svdq_gelu_bf16",
             "svdq_calib_absmax_cols", "svdq_calib_absmax_rows", "svdq_calib_smooth", "svdq_calib_scale_rows",
-            "svdq_calib_act_amax")
+            "svdq_calib_act_amax", "svdq_map_cache_stats")
 
 
 class SVDQError(RuntimeError):
@@ -105,6 +105,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                        ("svdq_calib_act_amax", [_P, _I64, _I64, _P, _P, _I, _P])):
         getattr(lib, name).restype = _I
         getattr(lib, name).argtypes = args
+    lib.svdq_map_cache_stats.restype = None
+    lib.svdq_map_cache_stats.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
     lib.svdq_get_device_error.restype = _I
     lib.svdq_get_device_error.argtypes = [_P, ctypes.POINTER(_I)]
     _lib = lib
@@ -243,6 +245,13 @@ def svdq_calib_act_amax(X, M, K, inv_s, amax, accumulate=False, stream=None) -> 
     _check(load_library().svdq_calib_act_amax(_ptr(X, torch.bfloat16, "X"), M, K, _ptr(inv_s, torch.float32, "inv_s"),
                                               _ptr(amax, torch.float32, "amax"), int(bool(accumulate)),
                                               _stream(stream)), "svdq_calib_act_amax")
+
+
+def svdq_map_cache_stats():
+    """(hits, misses) of the library's tensor-map cache."""
+    h, m = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    load_library().svdq_map_cache_stats(ctypes.byref(h), ctypes.byref(m))
+    return int(h.value), int(m.value)
 
 
 def svdq_version() -> int:
