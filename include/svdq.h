@@ -76,7 +76,8 @@ typedef enum {
     SVDQ_ERR_CUDA = 4,               /* a CUDA runtime/driver call or launch failed    */
     SVDQ_ERR_TIMEOUT = 5,            /* a kernel's bounded wait ran out (device error) */
     SVDQ_ERR_DEVICE = 6,             /* current device is not compute capability 10.x  */
-    SVDQ_ERR_SCRATCH = 7             /* shape needs more than the library's own scratch */
+    SVDQ_ERR_SCRATCH = 7,            /* shape needs more than the library's own scratch */
+    SVDQ_ERR_CHECK = 8               /* debug build: a copy failed its bounds/alignment check */
 } svdq_status;
 
 /* Human-readable name of a status code (static string). */
@@ -420,10 +421,25 @@ SVDQ_API void svdq_map_cache_stats(uint64_t* hits, uint64_t* misses);
 SVDQ_API svdq_status svdq_get_device_error(svdq_stream_t stream, int* site);
 
 /*
+ * svdq_build_flags -- bit 0 set in the debug build (libsvdq_check.so, compiled
+ * with -DSVDQ_CHECK): every TMA / bulk copy of the kernels is checked before it
+ * is issued (innermost coordinate aligned to 16 bytes, coordinates and sources
+ * inside their tensors, destination inside the launch's shared memory); a
+ * failed check skips the copy and records SVDQ_ERR_CHECK with the check's site
+ * (read by svdq_get_device_error; the kernel's bounded waits then end it).
+ * The pages have no counterpart (it is a debugging aid).
+ */
+SVDQ_API int svdq_build_flags(void);
+
+/*
  * svdq_linear_debug -- svdq_linear with test hooks, for the fault-path tests.
  *   debug_flags bit 0: the load warp issues no loads, so the MMA warp's first
- *                      wait can never complete and must run out.  Any other
- *                      bit is SVDQ_ERR_INVALID_ARG.
+ *                      wait can never complete and must run out.
+ *               bit 1: (debug build only) the first A box of every tile is
+ *                      requested at a misaligned innermost coordinate; the
+ *                      build's copy check skips it and records SVDQ_ERR_CHECK.
+ *                      SVDQ_ERR_INVALID_ARG in the regular build.
+ *   Any other bit is SVDQ_ERR_INVALID_ARG.
  *   timeout_ns: bound of every barrier wait (0 = the default of 2 s).
  * Otherwise identical to svdq_linear.
  */

@@ -39,18 +39,19 @@ def sources():
     return files + [os.path.join(ROOT, "include", "svdq.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(OUT):
+OUT_CHECK = os.path.join(PKG_DIR, "libsvdq_check.so")
+
+
+def up_to_date(out: str = OUT) -> bool:
+    if not os.path.exists(out):
         return False
-    t = os.path.getmtime(OUT)
+    t = os.path.getmtime(out)
     return all(os.path.getmtime(f) <= t for f in sources())
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and up_to_date():
-        return OUT
+def _compile(out: str, extra, verbose: bool) -> str:
     cmd = [nvcc_path(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "-Xptxas=-v", "-o", OUT + ".tmp", SRC]
+           "-Xcompiler", "-fvisibility=hidden", "-Xptxas=-v", *extra, "-o", out + ".tmp", SRC]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
@@ -59,11 +60,19 @@ def build(verbose: bool = False, force: bool = False) -> str:
     for kernel in ("8k_linearILb0E", "8k_linearILb1E"):
         regs = entry_registers(res.stdout + res.stderr, kernel)
         if regs != LINEAR_ENTRY_REGS:
-            os.remove(OUT + ".tmp")
+            os.remove(out + ".tmp")
             raise RuntimeError(f"{kernel} compiled to {regs} registers per thread at entry, expected "
                                f"{LINEAR_ENTRY_REGS}: its setmaxnreg split would not add up")
-    os.replace(OUT + ".tmp", OUT)
-    return OUT
+    os.replace(out + ".tmp", out)
+    return out
+
+
+def build(verbose: bool = False, force: bool = False, check: bool = False) -> str:
+    """Build libsvdq.so (check=True: the debug build libsvdq_check.so, every copy checked)."""
+    out = OUT_CHECK if check else OUT
+    if not force and up_to_date(out):
+        return out
+    return _compile(out, ["-DSVDQ_CHECK"] if check else [], verbose)
 
 
 def entry_registers(ptxas_log: str, kernel: str) -> int | None:
@@ -79,4 +88,4 @@ def entry_registers(ptxas_log: str, kernel: str) -> int | None:
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv, force=True))
+    print(build(verbose="--verbose" in sys.argv, force=True, check="--check" in sys.argv))

@@ -18,14 +18,34 @@ namespace svdq {
 __device__ unsigned int g_err_flags;
 __device__ unsigned int g_err_site;
 
-enum : unsigned { ERR_TIMEOUT = 1u };
+enum : unsigned { ERR_TIMEOUT = 1u, ERR_CHECK = 2u };
 
 SVDQ_DEV void report_timeout(unsigned site) {
-  atomicOr(&g_err_flags, ERR_TIMEOUT);
-  atomicExch(&g_err_site, site);
+  // a failed copy check (which makes later waits run out) keeps its own site
+  if (!(atomicOr(&g_err_flags, ERR_TIMEOUT) & ERR_CHECK)) atomicExch(&g_err_site, site);
 }
 
+// Debug build (-DSVDQ_CHECK, libsvdq_check.so): every TMA and bulk copy is checked before it is issued
+// (alignment of the innermost coordinate, coordinates and sources inside their tensors, destination
+// inside the launch's shared memory); a failed check records ERR_CHECK and the copy is skipped, so
+// the kernel's bounded waits end it with the error word set instead of issuing a faulting copy.
+SVDQ_DEV void report_check(unsigned site) {
+  atomicOr(&g_err_flags, ERR_CHECK);
+  atomicExch(&g_err_site, site);
+}
+#ifdef SVDQ_CHECK
+#define SVDQ_CHECK_OK(cond, site) ((cond) || (::svdq::report_check(site), false))
+#else
+#define SVDQ_CHECK_OK(cond, site) true
+#endif
+
 // --------------------------------------------------------------- basics -----
+SVDQ_DEV uint32_t dyn_smem_bytes() {
+  uint32_t v;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+  return v;
+}
+
 SVDQ_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

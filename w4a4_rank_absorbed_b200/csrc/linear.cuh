@@ -79,7 +79,10 @@ static_assert(LN_STAGES * LN_STREAMS <= 32 && LN_STREAMS == 3, "one lane per slo
 static_assert(LN_REGS_LOW * 256 + LN_REGS_HIGH * 256 == LN_THREADS * 128, "register split = launch budget");
 
 // Test hook (svdq_linear_debug): the load warp issues nothing, so the first wait must run out.
-enum : int { LN_DBG_NO_LOADS = 1 };
+// Test hooks (svdq_linear_debug): the load warp issues nothing, so the first wait must run out; or
+// (accepted by the check build only) the first A box of every tile is asked for at a misaligned
+// innermost coordinate, which the build's copy checks must catch.
+enum : int { LN_DBG_NO_LOADS = 1, LN_DBG_MISALIGN = 2 };
 
 #ifndef LN_RASTER_GM
 #define LN_RASTER_GM 12
@@ -369,10 +372,14 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
               const CUtensorMap* map = k == 0 ? (lr ? &tm_las : &tm_xq) : (lr ? &tm_l2p : &tm_wq);
               uint8_t* dst = k == 0 ? sA + stage * LN_A_BYTES
                                     : sB + stage * LN_B_BYTES + (k - 1) * (lr ? LN_LR_B_HALF : LN_B_HALF);
-              const int x = lr ? (kt - nkt) * (k == 0 ? 64 : 32) : kt * 128;
+              const int x = (lr ? (kt - nkt) * (k == 0 ? 64 : 32) : kt * 128) +
+                            ((args.debug & LN_DBG_MISALIGN) && k == 0 && kt == 0 ? 8 : 0);
               const int y = k == 0 ? mb * LN_BM : nb * LN_BN + (k - 1) * 128;
               __syncwarp(smask);
-              tma_load_2d(dst, map, &full[stage], x, y);
+              const uint32_t box = k == 0 ? (lr ? LN_A_BYTES : LN_A_BYTES) : (lr ? LN_LR_B_HALF : LN_B_HALF);
+              if (SVDQ_CHECK_OK((x * (lr ? 2 : 1)) % 16 == 0 && x >= 0 && y >= 0 &&
+                                    (uint32_t)(dst - smem_raw) + box <= dyn_smem_bytes(), 0x3c1))
+                tma_load_2d(dst, map, &full[stage], x, y);
               issued = true;
               last_parity = phase;
             }
@@ -394,7 +401,11 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
               uint8_t* dst = k == 0 ? sSFA + stage * LN_SFA_BYTES : sSFB + stage * LN_SFB_BYTES + 2048 * (k - 1);
               const uint8_t* src = k == 0 ? args.SFx + ((int64_t)mb * KAs + per * kt) * 512
                                           : args.SFw + ((int64_t)(2 * nb + k - 1) * KAs + per * kt) * 512;
-              bulk_load(dst, src, (uint32_t)(ka * 512), &sf_full[stage]);
+              const int64_t blocks = k == 0 ? sfx_blocks : sfw_blocks;
+              const int64_t atom = k == 0 ? (int64_t)mb * KAs + per * kt : (int64_t)(2 * nb + k - 1) * KAs + per * kt;
+              if (SVDQ_CHECK_OK(ka > 0 && atom + ka <= blocks * KAs && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
+                                    (uint32_t)(dst - smem_raw) + ka * 512 <= dyn_smem_bytes(), 0x3c2))
+                bulk_load(dst, src, (uint32_t)(ka * 512), &sf_full[stage]);
               issued = true;
               last_parity = phase;
             }

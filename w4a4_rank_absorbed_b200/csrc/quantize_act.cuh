@@ -245,14 +245,16 @@ __global__ void __launch_bounds__(QB_THREADS, 1) k_quantize_act(
         uint8_t* st = smem + s * Cfg::kStageBytes;
         const int c = 2 * (u_begin + i);                       // first chunk of the stage
         const bool pair = c + 1 < nch;
+        const bool fits = SVDQ_CHECK_OK(c >= 0 && c < nch && m0 >= 0 && m0 < Mpad &&
+                                            (uint32_t)(st - smem_raw) + Cfg::kStageBytes <= dyn_smem_bytes(), 0x2c1);
         if (xw) {
           mbar_arrive_expect_tx(&full[s], (uint32_t)((pair ? 2 : 1) * Cfg::kXTile));
-          if (pair) tma_load_3d(st, &tm_x, &full[s], 0, m0, c);
-          else tma_load_2d(st, &tm_x1, &full[s], c * QB_CHUNK, m0);
+          if (fits && pair) tma_load_3d(st, &tm_x, &full[s], 0, m0, c);
+          else if (fits) tma_load_2d(st, &tm_x1, &full[s], c * QB_CHUNK, m0);
         } else {
           mbar_arrive_expect_tx(&full[s], (uint32_t)((pair ? 2 : 1) * Cfg::kLTile));
-          if (pair) tma_load_3d(st + Cfg::kXBytes, &tm_l1, &full[s], 0, 0, c);
-          else tma_load_2d(st + Cfg::kXBytes, &tm_l11, &full[s], c * QB_CHUNK, 0);
+          if (fits && pair) tma_load_3d(st + Cfg::kXBytes, &tm_l1, &full[s], 0, 0, c);
+          else if (fits) tma_load_2d(st + Cfg::kXBytes, &tm_l11, &full[s], c * QB_CHUNK, 0);
         }
         issued = i + 1;
       }

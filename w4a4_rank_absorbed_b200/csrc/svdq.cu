@@ -455,6 +455,7 @@ const char* svdq_status_string(int status) {
     case SVDQ_ERR_TIMEOUT: return "SVDQ_ERR_TIMEOUT";
     case SVDQ_ERR_DEVICE: return "SVDQ_ERR_DEVICE";
     case SVDQ_ERR_SCRATCH: return "SVDQ_ERR_SCRATCH";
+    case SVDQ_ERR_CHECK: return "SVDQ_ERR_CHECK";
     default: return "SVDQ_ERR_UNKNOWN";
   }
 }
@@ -766,7 +767,11 @@ svdq_status svdq_linear_debug(const uint8_t* Xq, const uint8_t* SFx, float gs_x,
                               const uint8_t* SFw, float gs_w, const uint16_t* LAs, const uint16_t* L2p, int r,
                               const uint16_t* bias, void* Y, int y_fp32, int64_t M, int64_t N, int64_t K,
                               int debug_flags, uint64_t timeout_ns, svdq_stream_t stream) {
-  if (debug_flags & ~LN_DBG_NO_LOADS) return SVDQ_ERR_INVALID_ARG;
+#ifdef SVDQ_CHECK
+  if (debug_flags & ~(LN_DBG_NO_LOADS | LN_DBG_MISALIGN)) return SVDQ_ERR_INVALID_ARG;
+#else
+  if (debug_flags & ~LN_DBG_NO_LOADS) return SVDQ_ERR_INVALID_ARG;   // the misaligned box only where checked
+#endif
   return linear_impl(Xq, SFx, gs_x, Wq, SFw, gs_w, LAs, L2p, r, bias, Y, y_fp32, M, N, K, debug_flags, timeout_ns,
                      reinterpret_cast<cudaStream_t>(stream));
 }
@@ -780,7 +785,16 @@ svdq_status svdq_get_device_error(svdq_stream_t stream, int* site) {
       cudaMemcpyToSymbol(svdq::g_err_site, &zero, sizeof(zero)) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   if (site) *site = (int)where;
+  if (flags & svdq::ERR_CHECK) return SVDQ_ERR_CHECK;
   return (flags & svdq::ERR_TIMEOUT) ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+}
+
+int svdq_build_flags(void) {
+#ifdef SVDQ_CHECK
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 }  // extern "C"

@@ -16,6 +16,16 @@ import torch
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG_DIR, "libsvdq.so")
+CHECK_LIB_PATH = os.path.join(_PKG_DIR, "libsvdq_check.so")   # debug build: every copy checked
+
+
+def default_library_path() -> str:
+    """libsvdq.so, or the library named by the SVDQ_LIBRARY environment variable ("check" selects the
+    debug build libsvdq_check.so)."""
+    v = os.environ.get("SVDQ_LIBRARY", "")
+    if not v:
+        return LIB_PATH
+    return CHECK_LIB_PATH if v == "check" else v
 
 SVDQ_OK = 0
 SVDQ_ERR_INVALID_ARG = 1
@@ -25,6 +35,7 @@ SVDQ_ERR_CUDA = 4
 SVDQ_ERR_TIMEOUT = 5
 SVDQ_ERR_DEVICE = 6
 SVDQ_ERR_SCRATCH = 7
+SVDQ_ERR_CHECK = 8
 
 EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_weight", "svdq_quantize_act",
             "svdq_linear", "svdq_lowrank_down", "svdq_lowrank_up", "svdq_get_device_error", "svdq_linear_debug",
@@ -32,7 +43,7 @@ EXPORTED = ("svdq_status_string", "svdq_version", "svdq_sf_bytes", "svdq_pack_we
             "svdq_mx_sf_bytes", "svdq_pack_weight_mx", "svdq_quantize_act_mx", "svdq_linear_mx",
             "svdq_linear_gelu_quantize", "svdq_linear_gelu_quantize_workspace_bytes", "svdq_gelu_bf16",
             "svdq_calib_absmax_cols", "svdq_calib_absmax_rows", "svdq_calib_smooth", "svdq_calib_scale_rows",
-            "svdq_calib_act_amax", "svdq_map_cache_stats")
+            "svdq_calib_act_amax", "svdq_map_cache_stats", "svdq_build_flags")
 
 
 class SVDQError(RuntimeError):
@@ -49,11 +60,12 @@ _I = ctypes.c_int
 _F = ctypes.c_float
 
 
-def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     """Load libsvdq.so (raises if it has not been built)."""
     global _lib
     if _lib is not None:
         return _lib
+    path = path or default_library_path()
     if not os.path.exists(path):
         raise ImportError(f"CUDA library not built: {path} (run python -m w4a4_rank_absorbed_b200.build)")
     lib = ctypes.CDLL(path)
@@ -105,6 +117,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                        ("svdq_calib_act_amax", [_P, _I64, _I64, _P, _P, _I, _P])):
         getattr(lib, name).restype = _I
         getattr(lib, name).argtypes = args
+    lib.svdq_build_flags.restype = _I
+    lib.svdq_build_flags.argtypes = []
     lib.svdq_map_cache_stats.restype = None
     lib.svdq_map_cache_stats.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
     lib.svdq_get_device_error.restype = _I
@@ -252,6 +266,10 @@ def svdq_map_cache_stats():
     h, m = ctypes.c_uint64(0), ctypes.c_uint64(0)
     load_library().svdq_map_cache_stats(ctypes.byref(h), ctypes.byref(m))
     return int(h.value), int(m.value)
+
+
+def svdq_build_flags() -> int:
+    return int(load_library().svdq_build_flags())
 
 
 def svdq_version() -> int:
