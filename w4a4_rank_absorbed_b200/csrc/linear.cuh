@@ -586,6 +586,13 @@ __global__ void __launch_bounds__(LN_THREADS, 1) k_linear(
 
       const int row = mb * LN_BM + 32 * q + lane;
       const int n0 = nb * LN_BN + h * 128;
+      // The down-projection's B operand for these 128 columns (r2 rows of L1f2^T, 256 bytes each) into
+      // L1 now, so its fragment loads after the GELU hit L1 instead of waiting on L2.
+      if (lane < r2) {
+        const uint16_t* bl = args.L1fT2 + (int64_t)lane * N + n0;
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(bl));
+        if (n0 + 64 < N) asm volatile("prefetch.global.L1 [%0];" ::"l"(bl + 64));
+      }
       uint32_t p[64];                                // y, then x2 (bf16 pairs): p[8g + j] = columns 16g + 2j, +1
       uint32_t cw[4];                                // codes of two groups of 16 (two words each)
       uint32_t sw[2] = {0u, 0u};                     // scale words (4 groups each)
