@@ -43,7 +43,9 @@
  *     svdq_get_device_error().
  *   - Pointers must be 16-byte aligned (svdq_linear stores Y 32 bytes at a time
  *     when Y is 32-byte aligned, 16 bytes otherwise).  Shapes: K % 64 == 0,
- *     N % 16 == 0, r % 16 == 0 with 0 <= r <= 128, 1 <= M, K, N < 2^31.  Any M.
+ *     N % 16 == 0, r % 16 == 0 with 0 <= r <= 128, 1 <= K, N < 2^31, 0 <= M < 2^31.
+ *     M = 0 (an empty batch) is a valid call of every per-forward entry point: it
+ *     launches nothing and returns SVDQ_OK (buffer pointers may then be NULL).
  *   - Buffer sizes cannot be checked from pointers: every buffer must hold the
  *     shape the call states (a larger r than LAs / L2p were sized for makes the
  *     kernels read past them).

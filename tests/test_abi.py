@@ -61,7 +61,8 @@ def test_argument_errors_before_any_launch(lib):
     assert _linear(lib, N=24) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
     assert _linear(lib, r=8) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
     assert _linear(lib, r=144) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
-    assert _linear(lib, M=0) == svdq.SVDQ_ERR_INVALID_ARG
+    assert _linear(lib, M=-1) == svdq.SVDQ_ERR_INVALID_ARG
+    assert _linear(lib, M=0) == svdq.SVDQ_OK                 # an empty batch launches nothing
     assert _linear(lib, M=1 << 31) == svdq.SVDQ_ERR_UNSUPPORTED_SHAPE
     assert _linear(lib, Xq=None) == svdq.SVDQ_ERR_INVALID_ARG
     assert _linear(lib, LAs=None) == svdq.SVDQ_ERR_INVALID_ARG
@@ -95,3 +96,27 @@ def test_valid_arguments_without_a_gpu_report_a_device_error(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _linear(lib) in (svdq.SVDQ_ERR_CUDA, svdq.SVDQ_ERR_DEVICE)
+
+
+def test_empty_batch_is_a_no_op_and_shape_errors_still_apply():
+    """M = 0 launches nothing (no CUDA call, so this runs without a GPU) and returns SVDQ_OK with NULL
+    buffers; shape errors of the other dimensions are still reported."""
+    from w4a4_rank_absorbed_b200 import svdq as C
+    lib = C.load_library()
+    OK, UNSUP, INVAL = C.SVDQ_OK, C.SVDQ_ERR_UNSUPPORTED_SHAPE, C.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_quantize_act(None, 0, 256, None, 1.0, None, 32, 1.0, None, None, None, None, 0, None) == OK
+    assert lib.svdq_quantize_act(None, 0, 100, None, 1.0, None, 32, 1.0, None, None, None, None, 0, None) == UNSUP
+    assert lib.svdq_quantize_act_noalloc(None, 0, 256, None, 1.0, None, 16, 1.0, None, None, None, None) == OK
+    assert lib.svdq_linear(None, None, 1.0, None, None, 1.0, None, None, 32, None, None, 0, 0, 512, 256, None) == OK
+    assert lib.svdq_linear(None, None, 1.0, None, None, 1.0, None, None, 32, None, None, 0, 0, 500, 256, None) == UNSUP
+    assert lib.svdq_lowrank_down(None, 0, 256, None, 32, 1.0, None, None, 0, None) == OK
+    assert lib.svdq_lowrank_down(None, 0, 256, None, 0, 1.0, None, None, 0, None) == INVAL
+    assert lib.svdq_lowrank_up(None, None, 32, 1.0, None, 0, 0, 512, None) == OK
+    assert lib.svdq_quantize_act_mx(None, 0, 256, None, None, 0, 1.0, None, None, None, None, 0, None) == OK
+    assert lib.svdq_quantize_act_mx(None, 0, 192, None, None, 0, 1.0, None, None, None, None, 0, None) == UNSUP
+    assert lib.svdq_linear_mx(None, None, None, None, None, None, 0, None, None, 0, 0, 256, 192, None) == UNSUP
+    assert lib.svdq_linear_gelu_quantize(None, None, 1.0, None, None, 1.0, None, None, 0, None, 0, 512, 256, None,
+                                         1.0, None, 32, 1.0, None, None, None, None, 0, None) == OK
+    assert lib.svdq_linear_gelu_quantize(None, None, 1.0, None, None, 1.0, None, None, 0, None, 0, 512, 256, None,
+                                         1.0, None, 48, 1.0, None, None, None, None, 0, None) == UNSUP
+    assert lib.svdq_quantize_act(None, -1, 256, None, 1.0, None, 0, 1.0, None, None, None, None, 0, None) == INVAL

@@ -184,8 +184,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
+// M = 0 (an empty batch) passes; the per-forward entry points then return SVDQ_OK at once.
 svdq_status check_shape(int64_t M, int64_t N, int64_t K, int r) {
-  if (M < 1 || N < 1 || K < 1 || r < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0 || N < 1 || K < 1 || r < 0) return SVDQ_ERR_INVALID_ARG;
   if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (K % 64 != 0 || N % 16 != 0 || r % 16 != 0 || r > 128) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   return SVDQ_OK;
@@ -353,6 +354,8 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   // gq: no Y; the epilogue writes the next layer's quantized activations instead.
   svdq_status st = check_shape(M, N, y_accum ? 64 : K, r);
   if (st != SVDQ_OK) return st;
+  if (M == 0)                                 // an empty batch: nothing to launch
+    return (y_accum && r == 0) ? SVDQ_ERR_INVALID_ARG : (mx && K % 128 != 0) ? SVDQ_ERR_UNSUPPORTED_SHAPE : SVDQ_OK;
   if (y_accum ? (r == 0 || !LAs || !L2p || !Y || bias)
               : (!Xq || !SFx || !Wq || !SFw || (!gq && !Y) || (r > 0 && (!LAs || !L2p))))
     return SVDQ_ERR_INVALID_ARG;
@@ -529,6 +532,7 @@ svdq_status svdq_quantize_act_mx(const uint16_t* X, int64_t M, int64_t K, const 
   svdq_status st = check_shape(M, 16, K, r);
   if (st != SVDQ_OK) return st;
   if (K % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;                 // an empty batch: nothing to launch
   if (!X || !inv_s || !Xq || !SFx || (r > 0 && (!L1fT || !LAs))) return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!workspace || workspace_bytes < qa_workspace_bytes(M, r))) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(inv_s) || !aligned16(Xq) || !aligned16(SFx) ||
@@ -562,6 +566,7 @@ svdq_status svdq_linear_gelu_quantize(const uint8_t* Xq, const uint8_t* SFx, flo
   svdq_status st = check_shape(M, N, K, r);
   if (st != SVDQ_OK) return st;
   if (N % 64 != 0 || (r2 != 0 && r2 != 16 && r2 != 32)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;                 // an empty batch: nothing to launch
   if (r2 > 0 && workspace_bytes < gq_workspace_bytes(M, N, r2)) return SVDQ_ERR_INVALID_ARG;
   GqArgs g;
   g.inv_s2 = inv_s2;
@@ -701,6 +706,7 @@ svdq_status svdq_quantize_act(const uint16_t* X, int64_t M, int64_t K, const flo
                               void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
   svdq_status st = check_shape(M, 16, K, r);
   if (st != SVDQ_OK) return st;
+  if (M == 0) return SVDQ_OK;                 // an empty batch: nothing to launch
   if (!X || !inv_s || !Xq || !SFx || (r > 0 && (!L1fT || !LAs))) return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!workspace || workspace_bytes < qa_workspace_bytes(M, r))) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(inv_s) || !aligned16(Xq) || !aligned16(SFx) ||
@@ -718,6 +724,7 @@ svdq_status svdq_quantize_act_noalloc(const uint16_t* X, int64_t M, int64_t K, c
                                       uint16_t* LAs, svdq_stream_t stream) {
   svdq_status st = check_shape(M, 16, K, r);
   if (st != SVDQ_OK) return st;
+  if (M == 0) return SVDQ_OK;                 // an empty batch: nothing to launch
   if (!X || !inv_s || !Xq || !SFx || (r > 0 && (!L1fT || !LAs))) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(inv_s) || !aligned16(Xq) || !aligned16(SFx) ||
       (r > 0 && (!aligned16(L1fT) || !aligned16(LAs))))
@@ -740,6 +747,7 @@ svdq_status svdq_lowrank_down(const uint16_t* X, int64_t M, int64_t K, const uin
                               uint16_t* LAs, void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
   svdq_status st = check_shape(M, 16, K, r);
   if (st != SVDQ_OK) return st;
+  if (M == 0) return r == 0 ? SVDQ_ERR_INVALID_ARG : SVDQ_OK;   // an empty batch: nothing to launch
   if (r == 0 || !X || !L1fT || !LAs || !workspace || workspace_bytes < qa_workspace_bytes(M, r))
     return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(L1fT) || !aligned16(LAs) || !aligned16(workspace)) return SVDQ_ERR_MISALIGNED;
