@@ -325,12 +325,14 @@ class Timer:
         torch.cuda.synchronize()
         return e0.elapsed_time(e1)
 
-    def per_launch(self, fn, n=GRAPH_LAUNCHES, reps=GRAPH_REPLAYS):
-        g = self.capture(fn, n)
-        g.replay()
-        self.torch.cuda.synchronize()
-        samples = [self.replay_ms(g) / n for _ in range(reps)]
-        del g
+    def per_launch(self, fn, n=GRAPH_LAUNCHES, reps=GRAPH_REPLAYS, name="graph"):
+        """Per-launch times of a graph of n launches replayed reps times (an NVTX range per leg)."""
+        with self.torch.cuda.nvtx.range(name):
+            g = self.capture(fn, n)
+            g.replay()
+            self.torch.cuda.synchronize()
+            samples = [self.replay_ms(g) / n for _ in range(reps)]
+            del g
         return samples
 
 
@@ -428,12 +430,12 @@ def measure_set(s, timer, dev, flush_buf):
     torch.cuda.synchronize()
     out = {}
     for key in ("step", "quantize", "gemm", "plain", "plain_qa", "plain_ln"):
-        out[key] = timer.per_launch(fns[key])
+        out[key] = timer.per_launch(fns[key], name=key)
     if r:
         for key in ("unfused", "down", "up"):
-            out[key] = timer.per_launch(fns[key])
+            out[key] = timer.per_launch(fns[key], name=key)
     # L2-warm: one layer copy over and over (its inputs, codes and weight stay in the L2 between steps).
-    out["step_l2_warm"] = timer.per_launch(lambda i: fns["step"](0))
+    out["step_l2_warm"] = timer.per_launch(lambda i: fns["step"](0), name="step_l2_warm")
     # L2-flushed: a 256 MB write before every step on one copy, minus the same writes alone.
     flush = lambda i: flush_buf.fill_(i & 0xFF)                       # noqa: E731
     both = timer.per_launch(lambda i: (flush(i), fns["step"](0)))
@@ -474,7 +476,7 @@ def mlp_chain_report(s1, s2, timer, dev):
         unfused(i)
         fused(i)
     torch.cuda.synchronize()
-    d = {k: stats(timer.per_launch(f)) for k, f in (("fused", fused), ("unfused", unfused),
+    d = {k: stats(timer.per_launch(f, name="mlp_" + k)) for k, f in (("fused", fused), ("unfused", unfused),
                                                      ("fc1_fused_gemm", fc1_fused_gemm), ("gelu", gelu_only))}
     K1, N1, r1 = s1["K"], s1["N"], s1["r"]
     N2, r2 = s2["N"], s2["r"]

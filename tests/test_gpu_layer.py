@@ -87,3 +87,23 @@ def test_tensor_maps_are_cached_across_calls():
     assert h1 - h0 == 4 * n                      # Xq, Wq, LAs, L2p maps of every call
     print(f"svdq_linear host time per call through ctypes, cached maps: {(t1 - t0) / n * 1e6:.1f} us")
     g.check_errors()
+
+
+def test_packed_layer_state_round_trip(tmp_path):
+    """A packed layer saved with torch.save and rebuilt without packing gives identical outputs."""
+    from w4a4_rank_absorbed_b200.calib import calibrate
+    from w4a4_rank_absorbed_b200.layer import SVDQLinear
+    wl = small_case(300, 512, 384, 32, seed=21)
+    L = SVDQLinear(calibrate(wl.X, wl.W, 32, wl.alpha, bias=wl.bias))
+    X = bf16_dev(wl.X)
+    Y0 = L.forward(X)
+    path = tmp_path / "layer.pt"
+    torch.save(L.state_dict(), path)
+    L2 = SVDQLinear.from_state_dict(torch.load(path), device="cuda")
+    Y1 = L2.forward(X)
+    torch.cuda.synchronize()
+    assert torch.equal(Y0, Y1)
+    with pytest.raises(ValueError):
+        bad = L.state_dict()
+        bad["Wq"] = bad["Wq"][:, :10]
+        SVDQLinear.from_state_dict(bad, device="cuda")

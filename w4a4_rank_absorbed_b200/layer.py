@@ -68,6 +68,41 @@ class SVDQLinear:
         self.lr_scale = _f32(1.0 / (np.float64(self.gs_x) * np.float64(self.gs_w)))
         self._act: Dict[int, tuple] = {}
 
+    # ------------------------------------------------------------ checkpoint --
+    _PACKED = ("Wq", "SFw", "gs_w_dev", "L2p", "inv_s", "L1fT", "bias")
+
+    def state_dict(self) -> Dict[str, object]:
+        """The packed layer as plain tensors (host copies) and scalars: save it with torch.save and
+        rebuild with SVDQLinear.from_state_dict without packing the weight again."""
+        out: Dict[str, object] = {"K": self.K, "N": self.N, "r": self.r, "gs_x": self.gs_x, "gs_w": self.gs_w,
+                                  "lr_scale": self.lr_scale}
+        for k in self._PACKED:
+            t = getattr(self, k)
+            out[k] = None if t is None else t.detach().cpu()
+        return out
+
+    @classmethod
+    def from_state_dict(cls, state: Dict[str, object], device: Optional[torch.device] = None) -> "SVDQLinear":
+        """A layer from state_dict() output, its buffers copied to `device` (no packing kernel runs)."""
+        self = cls.__new__(cls)
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        self.K, self.N, self.r = int(state["K"]), int(state["N"]), int(state["r"])
+        self.gs_x, self.gs_w, self.lr_scale = float(state["gs_x"]), float(state["gs_w"]), float(state["lr_scale"])
+        for k in cls._PACKED:
+            t = state[k]
+            setattr(self, k, None if t is None else t.to(dev).contiguous())
+        expect = {"Wq": (self.N, self.K // 2), "L2p": (self.N, self.r) if self.r else None,
+                  "inv_s": (self.K,), "L1fT": (self.r, self.K) if self.r else None}
+        for k, shape in expect.items():
+            t = getattr(self, k)
+            if (shape is None) != (t is None) or (t is not None and tuple(t.shape) != shape):
+                raise ValueError(f"state entry {k} has shape {None if t is None else tuple(t.shape)}, expected {shape}")
+        if self.SFw.numel() != _C.svdq_sf_bytes(self.N, self.K):
+            raise ValueError("state entry SFw has the wrong size")
+        self._act = {}
+        return self
+
     def act_buffers(self, M: int):
         """Device buffers of the quantized activations for M rows (allocated once per M): Xq, SFx, LAs."""
         return self._act_set(M)[:3]
