@@ -10,7 +10,7 @@ from oracle import decompose as OD
 from oracle import linear as OL
 from oracle.layout import sf_to_storage
 
-# Tolerances of the layer output against the float64 oracle (the benchmark spec's bounds):
+# Tolerances of the layer output against the float64 oracle (the stated output tolerances):
 REL_FRO = 2e-3          # ||Y - Y_or||_F / ||Y_or||_F
 MAX_ABS_RMS = 1e-2      # max |Y - Y_or| <= 1e-2 rms(Y_or)   (+ half a bf16 ulp of Y_or for bf16 output)
 LA_REL = 2e-5           # |LAs_hi + LAs_lo - lr_scale X L1f| <= 2e-5 lr_scale (|X| |L1f|)
