@@ -47,14 +47,16 @@ readings taken here:
       -> x2 = bf16(gelu_f32(y1)) -> fc2's activation quantization and
       low-rank down-projection (oracle.linear.quantize_act) -> fc2's layer.
 
-Pins (tests/test_oracle_mlp.py): exp against the float64 exponential over
-[-80, 0] (relative error within a few float32 ulp); the reciprocal against
-1/d over [1, 2] (within 1.5 float32 ulp); gelu_f32 against the
-float64 closed form over every finite bf16 input; the closed form's
-constants against torch's float64 GELU (tanh approximation); GELU(1) against
-its decimal value; GELU(0) = 0 and GELU(-0) = -0; the odd-part identity
-GELU(y) - GELU(-y) = y; the chain against its parts on a tiny case computed
-element by element.
+Pins (tests/test_oracle_mlp.py): fma32 against the exact rational value
+rounded once (random triples, binary32 midpoints approached from both sides,
+subnormal results); exp against the float64 exponential over [-80, 0]
+(within 4 float32 ulp); the reciprocal against 1/d over [1, 2] (within 1.5
+ulp); gelu_f32 against the float64 logistic form over every finite bf16 input
+(the bound grows with |t|, since exp(-|t|) magnifies the rounding of t); the
+logistic form against the tanh closed form and torch's float64 GELU (tanh
+approximation); GELU(+-1) against their decimal values; GELU(0) = 0 and
+GELU(-0) = -0; the odd-part identity GELU(y) - GELU(-y) = y; the chain
+against its parts on a tiny case computed element by element.
 """
 from __future__ import annotations
 
