@@ -120,3 +120,25 @@ def test_empty_batch_is_a_no_op_and_shape_errors_still_apply():
     assert lib.svdq_linear_gelu_quantize(None, None, 1.0, None, None, 1.0, None, None, 0, None, 0, 512, 256, None,
                                          1.0, None, 48, 1.0, None, None, None, None, 0, None) == UNSUP
     assert lib.svdq_quantize_act(None, -1, 256, None, 1.0, None, 0, 1.0, None, None, None, None, 0, None) == INVAL
+
+
+def test_plain_c_client_compiles_against_the_header_and_runs(tmp_path):
+    """include/svdq.h compiles as strict C99 and a C program linked to libsvdq.so gets the documented
+    answers from the calls that need no GPU (sizes, argument errors, empty batches)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    from w4a4_rank_absorbed_b200 import svdq
+    svdq.load_library()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib_dir = os.path.dirname(svdq.LIB_PATH)
+    exe = str(tmp_path / "svdq_client")
+    build = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                            "-I", os.path.join(root, "include"), os.path.join(root, "tests", "c_client", "svdq_client.c"),
+                            "-L", lib_dir, "-l:libsvdq.so", "-Wl,-rpath," + lib_dir, "-o", exe],
+                           capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and "c client ok" in run.stdout, run.stdout + run.stderr

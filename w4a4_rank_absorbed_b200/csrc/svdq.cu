@@ -354,8 +354,8 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
   // gq: no Y; the epilogue writes the next layer's quantized activations instead.
   svdq_status st = check_shape(M, N, y_accum ? 64 : K, r);
   if (st != SVDQ_OK) return st;
-  if (M == 0)                                 // an empty batch: nothing to launch
-    return (y_accum && r == 0) ? SVDQ_ERR_INVALID_ARG : (mx && K % 128 != 0) ? SVDQ_ERR_UNSUPPORTED_SHAPE : SVDQ_OK;
+  if (mx && K % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return (y_accum && r == 0) ? SVDQ_ERR_INVALID_ARG : SVDQ_OK;   // an empty batch: nothing to launch
   if (y_accum ? (r == 0 || !LAs || !L2p || !Y || bias)
               : (!Xq || !SFx || !Wq || !SFw || (!gq && !Y) || (r > 0 && (!LAs || !L2p))))
     return SVDQ_ERR_INVALID_ARG;
@@ -397,7 +397,6 @@ svdq_status linear_impl(const uint8_t* Xq, const uint8_t* SFx, float gs_x, const
     tm_xq = tm_las;
     tm_wq = tm_l2p;
   }
-  if (mx && K % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   const int variant = gq ? 2 : mx ? 1 : 0;
   auto kernel = gq ? k_linear<false, true> : mx ? k_linear<true, false> : k_linear<false, false>;
   const int smem_bytes = gq ? LN_SMEM_GQ : LN_SMEM;
